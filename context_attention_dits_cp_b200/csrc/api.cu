@@ -1,0 +1,446 @@
+// The C-ABI of libcpattn: argument validation, dispatch and the composite
+// (unified sequence parallelism) call.  Declarations and the contract of
+// every entry point are in include/cpattn.h.
+
+#include <cmath>
+#include <cstring>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace cpattn {
+
+// One error word per device (a __device__ variable exists once per device
+// the library's module is loaded on); kernels get its address.
+__device__ int g_device_error_word = 0;
+
+namespace {
+
+int* device_error_ptr() {
+  static int* ptrs[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error_word) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+// Byte range [lo, hi) a tensor's elements can touch.
+void byte_range(const TensorView& t, uintptr_t* lo, uintptr_t* hi) {
+  long long span = 0;
+  bool empty = false;
+  for (int i = 0; i < t.ndim; ++i) {
+    if (t.shape[i] == 0) empty = true;
+    span += (t.shape[i] - 1) * (t.stride[i] < 0 ? -t.stride[i] : t.stride[i]);
+  }
+  *lo = reinterpret_cast<uintptr_t>(t.data);
+  *hi = empty ? *lo : *lo + (uintptr_t)((span + 1) * dtype_size(t.dtype));
+}
+
+bool overlaps(const TensorView& a, const TensorView& b) {
+  uintptr_t a0, a1, b0, b1;
+  byte_range(a, &a0, &a1);
+  byte_range(b, &b0, &b1);
+  if (a0 == a1 || b0 == b1) return false;
+  return a0 < b1 && b0 < a1;
+}
+
+// A tensor with no elements may carry a NULL pointer; it is never read.
+int check_basic(const cp_tensor* t, int ndim) {
+  if (!t) return CP_ERR_NULL;
+  if (t->ndim != ndim) return CP_ERR_SHAPE;
+  if (t->dtype != CP_F32 && t->dtype != CP_BF16) return CP_ERR_DTYPE;
+  bool empty = false;
+  for (int i = 0; i < ndim; ++i) {
+    if (t->shape[i] < 0 || t->shape[i] > 0x7fffffffLL) return CP_ERR_SHAPE;
+    if (t->stride[i] < 0) return CP_ERR_ALIGN;
+    if (t->shape[i] == 0) empty = true;
+  }
+  if (!t->data && !empty) return CP_ERR_NULL;
+  return CP_OK;
+}
+
+// Element-stride / base alignment to `bytes` for every dim but the last,
+// which must be contiguous.
+int check_vector_layout(const cp_tensor* t, int bytes) {
+  const int es = dtype_size(t->dtype);
+  if (t->stride[t->ndim - 1] != 1 && t->shape[t->ndim - 1] > 1) return CP_ERR_ALIGN;
+  if (reinterpret_cast<uintptr_t>(t->data) % bytes) return CP_ERR_ALIGN;
+  for (int i = 0; i < t->ndim - 1; ++i)
+    if ((t->stride[i] * es) % bytes) return CP_ERR_ALIGN;
+  return CP_OK;
+}
+
+float resolve_scale(float scale, int64_t D) {
+  if (scale == 0.f || std::isnan(scale)) return 1.0f / std::sqrt((float)D);
+  return scale;
+}
+
+int launch_status(int st) { return st; }
+
+// Shared validation of attention arguments.  On success fills `a` (without
+// chunk offsets) and reports whether there is anything to compute.
+int prepare_attention(const cp_tensor* q, const cp_tensor* k, const cp_tensor* v, float scale,
+                      const cp_tensor* out, const cp_tensor* lse, bool lse_optional,
+                      RingArgs* a) {
+  int st;
+  if ((st = check_basic(q, 4)) || (st = check_basic(k, 4)) || (st = check_basic(v, 4)) ||
+      (st = check_basic(out, 4)))
+    return st;
+  if (!lse_optional || lse) {
+    if ((st = check_basic(lse, 3))) return st;
+    if (lse->dtype != CP_F32) return CP_ERR_DTYPE;
+  }
+  if (q->dtype != k->dtype || q->dtype != v->dtype) return CP_ERR_DTYPE;
+  const int64_t B = q->shape[0], Sq = q->shape[1], H = q->shape[2], D = q->shape[3];
+  const int64_t Skv = k->shape[1];
+  if (D != 64 && D != 128) return CP_ERR_SHAPE;
+  if (k->shape[0] != B || k->shape[2] != H || k->shape[3] != D) return CP_ERR_SHAPE;
+  for (int i = 0; i < 4; ++i)
+    if (v->shape[i] != k->shape[i]) return CP_ERR_SHAPE;
+  for (int i = 0; i < 4; ++i)
+    if (out->shape[i] != q->shape[i]) return CP_ERR_SHAPE;
+  if (lse && (lse->shape[0] != B || lse->shape[1] != H || lse->shape[2] != Sq))
+    return CP_ERR_SHAPE;
+  if (B * H * ((Sq + 255) / 256) > 0x7fffffffLL) return CP_ERR_SHAPE;
+  // q/k/v: the tensor-core path reads through TMA (16-byte base and strides)
+  if (q->dtype == CP_BF16) {
+    if ((st = check_vector_layout(q, 16)) || (st = check_vector_layout(k, 16)) ||
+        (st = check_vector_layout(v, 16)))
+      return st;
+  } else {
+    if ((st = check_vector_layout(q, 4)) || (st = check_vector_layout(k, 4)) ||
+        (st = check_vector_layout(v, 4)))
+      return st;
+  }
+  // out rows are written with 16-byte vector stores
+  if ((st = check_vector_layout(out, 16))) return st;
+  a->q = view_of(q);
+  a->k = view_of(k);
+  a->v = view_of(v);
+  a->out = view_of(out);
+  a->lse = view_of(lse);
+  if (overlaps(a->out, a->q) || overlaps(a->out, a->k) || overlaps(a->out, a->v))
+    return CP_ERR_ALIAS;
+  if (lse && (overlaps(a->lse, a->q) || overlaps(a->lse, a->k) || overlaps(a->lse, a->v) ||
+              overlaps(a->lse, a->out)))
+    return CP_ERR_ALIAS;
+  a->scale = resolve_scale(scale, D);
+  return CP_OK;
+}
+
+int run_attention(RingArgs& a, cudaStream_t stream) {
+  if (a.q.shape[1] == 0 || a.q.shape[0] == 0 || a.q.shape[2] == 0) return CP_OK;
+  a.dev_err = device_error_ptr();
+  if (!a.dev_err) return CP_ERR_CUDA;
+  const int64_t total = a.chunk_off[a.n_chunks] - a.chunk_off[0];
+  if (total == 0) return launch_fill_empty(a.out, a.lse, stream);
+  if (a.q.dtype == CP_BF16) return launch_attn_ring_tc(a, stream);
+  return launch_attn_ring_f32(a, stream);
+}
+
+int ring_impl(const cp_tensor* q, const cp_tensor* k, const cp_tensor* v,
+              const int64_t* chunk_offsets, int n_chunks, float scale, cp_tensor* out,
+              cp_tensor* lse, void* stream) {
+  RingArgs a;
+  int st = prepare_attention(q, k, v, scale, out, lse, true, &a);
+  if (st) return st;
+  if (!chunk_offsets) return CP_ERR_NULL;
+  if (n_chunks < 1 || n_chunks > CP_MAX_CHUNKS) return CP_ERR_OFFSETS;
+  if (chunk_offsets[0] != 0 || chunk_offsets[n_chunks] != k->shape[1]) return CP_ERR_OFFSETS;
+  for (int c = 0; c < n_chunks; ++c)
+    if (chunk_offsets[c + 1] < chunk_offsets[c]) return CP_ERR_OFFSETS;
+  a.chunk_off = chunk_offsets;
+  a.n_chunks = n_chunks;
+  return run_attention(a, as_stream(stream));
+}
+
+}  // namespace
+}  // namespace cpattn
+
+using namespace cpattn;
+
+extern "C" {
+
+int cp_attn_partial(const cp_tensor* q, const cp_tensor* k_chunk, const cp_tensor* v_chunk,
+                    float scale, cp_tensor* out, cp_tensor* lse, void* stream) {
+  RingArgs a;
+  int st = prepare_attention(q, k_chunk, v_chunk, scale, out, lse, false, &a);
+  if (st) return st;
+  const int64_t offs[2] = {0, k_chunk->shape[1]};
+  a.chunk_off = offs;
+  a.n_chunks = 1;
+  return run_attention(a, as_stream(stream));
+}
+
+int cp_ring_attention(const cp_tensor* q, const cp_tensor* k, const cp_tensor* v,
+                      const int64_t* chunk_offsets, int n_chunks, float scale, cp_tensor* out,
+                      cp_tensor* lse, void* stream) {
+  return ring_impl(q, k, v, chunk_offsets, n_chunks, scale, out, lse, stream);
+}
+
+int cp_lse_merge(cp_tensor* out_acc, cp_tensor* lse_acc, const cp_tensor* out_i,
+                 const cp_tensor* lse_i, void* stream) {
+  int st;
+  if ((st = check_basic(out_acc, 4)) || (st = check_basic(lse_acc, 3)) ||
+      (st = check_basic(out_i, 4)) || (st = check_basic(lse_i, 3)))
+    return st;
+  if (out_acc->dtype != CP_F32 || lse_acc->dtype != CP_F32 || lse_i->dtype != CP_F32)
+    return CP_ERR_DTYPE;
+  const int64_t B = out_acc->shape[0], S = out_acc->shape[1], H = out_acc->shape[2],
+                D = out_acc->shape[3];
+  if (D != 64 && D != 128) return CP_ERR_SHAPE;
+  for (int i = 0; i < 4; ++i)
+    if (out_i->shape[i] != out_acc->shape[i]) return CP_ERR_SHAPE;
+  const int64_t want[3] = {B, H, S};
+  for (int i = 0; i < 3; ++i)
+    if (lse_acc->shape[i] != want[i] || lse_i->shape[i] != want[i]) return CP_ERR_SHAPE;
+  // one lane moves D/32 consecutive elements with a single vector access
+  const int lane_bytes_acc = (int)(D / 32) * 4;
+  const int lane_bytes_in = (int)(D / 32) * dtype_size(out_i->dtype);
+  if ((st = check_vector_layout(out_acc, lane_bytes_acc)) ||
+      (st = check_vector_layout(out_i, lane_bytes_in)))
+    return st;
+  if ((st = check_vector_layout(lse_acc, 4)) || (st = check_vector_layout(lse_i, 4))) {
+    // lse may be strided in any dim; only natural alignment is needed
+    if (reinterpret_cast<uintptr_t>(lse_acc->data) % 4 ||
+        reinterpret_cast<uintptr_t>(lse_i->data) % 4)
+      return CP_ERR_ALIGN;
+  }
+  const TensorView va = view_of(out_acc), vla = view_of(lse_acc), vi = view_of(out_i),
+                   vli = view_of(lse_i);
+  if (overlaps(va, vi) || overlaps(va, vla) || overlaps(va, vli) || overlaps(vla, vi) ||
+      overlaps(vla, vli))
+    return CP_ERR_ALIAS;
+  if (B == 0 || S == 0 || H == 0) return CP_OK;
+  return launch_lse_merge(va, vla, vi, vli, as_stream(stream));
+}
+
+int cp_ulysses_permute(const cp_tensor* x, cp_tensor* y, int degree, int dir, void* stream) {
+  int st;
+  if ((st = check_basic(x, 5)) || (st = check_basic(y, 5))) return st;
+  if (x->dtype != y->dtype) return CP_ERR_DTYPE;
+  if (dir != 0 && dir != 1) return CP_ERR_SHAPE;
+  if (degree < 1) return CP_ERR_DEGREE;
+  const int64_t U = degree;
+  if (x->shape[0] != U || y->shape[0] != U) return CP_ERR_SHAPE;
+  const int64_t B = x->shape[1], D = x->shape[4];
+  if (y->shape[1] != B || y->shape[4] != D) return CP_ERR_SHAPE;
+  // seq-shard side [U, B, S/U, H, D] and head-shard side [U, B, S, H/U, D]
+  const cp_tensor* seq = dir == 0 ? x : y;
+  const cp_tensor* head = dir == 0 ? y : x;
+  const int64_t H = seq->shape[3], S = head->shape[2];
+  if (H % U || S % U) return CP_ERR_DEGREE;
+  if (seq->shape[2] * U != S || head->shape[3] * U != H) return CP_ERR_SHAPE;
+  // (heads, D) packed on both sides: every (rank, batch, token) run of H/U
+  // heads is contiguous
+  const cp_tensor* both[2] = {x, y};
+  for (const cp_tensor* t : both) {
+    if (t->shape[4] > 1 && t->stride[4] != 1) return CP_ERR_ALIGN;
+    if (t->shape[3] > 1 && t->stride[3] != D) return CP_ERR_ALIGN;
+  }
+  const TensorView vx = view_of(x), vy = view_of(y);
+  if (overlaps(vx, vy)) return CP_ERR_ALIAS;
+  return launch_ulysses_permute(vx, vy, degree, dir, as_stream(stream));
+}
+
+size_t cp_usp_workspace_bytes(int64_t B, int64_t S, int64_t H, int64_t D, int in_dtype,
+                              int out_dtype, int ring_degree, int ulysses_degree) {
+  if (B < 0 || S < 0 || H < 0 || D < 0 || ring_degree < 1 || ulysses_degree < 1) return 0;
+  if ((in_dtype != CP_F32 && in_dtype != CP_BF16) || (out_dtype != CP_F32 && out_dtype != CP_BF16))
+    return 0;
+  const size_t n = (size_t)B * S * H * D;   // elements of one full tensor
+  auto rnd = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  return 3 * rnd(n * dtype_size(in_dtype)) + rnd(n * dtype_size(out_dtype));
+}
+
+int cp_usp_attention(const cp_tensor* qs, const cp_tensor* ks, const cp_tensor* vs,
+                     int ring_degree, int ulysses_degree, float scale, void* workspace,
+                     size_t workspace_bytes, cp_tensor* outs, cp_tensor* lse, void* stream) {
+  int st;
+  if ((st = check_basic(qs, 5)) || (st = check_basic(ks, 5)) || (st = check_basic(vs, 5)) ||
+      (st = check_basic(outs, 5)))
+    return st;
+  if (qs->dtype != ks->dtype || qs->dtype != vs->dtype) return CP_ERR_DTYPE;
+  const int64_t R = ring_degree, U = ulysses_degree;
+  if (R < 1 || U < 1 || R * U > 4096) return CP_ERR_DEGREE;
+  const int64_t G = qs->shape[0], B = qs->shape[1], Sg = qs->shape[2], H = qs->shape[3],
+                D = qs->shape[4];
+  const cp_tensor* others[3] = {ks, vs, outs};
+  for (const cp_tensor* t : others)
+    for (int i = 0; i < 5; ++i)
+      if (t->shape[i] != qs->shape[i]) return CP_ERR_SHAPE;
+  if (G != R * U) return CP_ERR_DEGREE;
+  if (H % U) return CP_ERR_DEGREE;
+  const int64_t S = Sg * G, SR = Sg * U, Hg = H / U;
+  if (lse) {
+    if ((st = check_basic(lse, 3))) return st;
+    if (lse->dtype != CP_F32) return CP_ERR_DTYPE;
+    if (lse->shape[0] != B || lse->shape[1] != H || lse->shape[2] != S) return CP_ERR_SHAPE;
+  }
+  const size_t need =
+      cp_usp_workspace_bytes(B, S, H, D, qs->dtype, outs->dtype, ring_degree, ulysses_degree);
+  if (!workspace) return CP_ERR_WORKSPACE;
+  if (workspace_bytes < need) return CP_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return CP_ERR_ALIGN;
+  if (B == 0 || S == 0 || H == 0) return CP_OK;
+
+  const size_t n = (size_t)B * S * H * D;
+  auto rnd = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  const int esi = dtype_size(qs->dtype), eso = dtype_size(outs->dtype);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* Y[3] = {ws, ws + rnd(n * esi), ws + 2 * rnd(n * esi)};
+  uint8_t* Yo = ws + 3 * rnd(n * esi);
+  // Head-sharded buffers, [U, B, S, H/U, D] contiguous: tokens of ring block
+  // r sit at sequence offset r*S/R of every head group.
+  auto head_view = [&](uint8_t* base, int dt, int64_t r, int64_t len) {
+    cp_tensor t;
+    memset(&t, 0, sizeof(t));
+    t.dtype = dt;
+    t.ndim = 5;
+    const int64_t sh[5] = {U, B, len, Hg, D};
+    const int64_t sd[5] = {B * S * Hg * D, S * Hg * D, Hg * D, D, 1};
+    for (int i = 0; i < 5; ++i) {
+      t.shape[i] = sh[i];
+      t.stride[i] = sd[i];
+    }
+    t.data = base + (size_t)(r * SR * Hg * D) * dtype_size(dt);
+    return t;
+  };
+  auto shard_slice = [&](const cp_tensor* t, int64_t r) {
+    cp_tensor s = *t;
+    s.shape[0] = U;
+    s.data = static_cast<uint8_t*>(t->data) + (size_t)(r * U * t->stride[0]) * dtype_size(t->dtype);
+    return s;
+  };
+  const cp_tensor* ins[3] = {qs, ks, vs};
+  // 1. Ulysses all-to-all inside every ring group r
+  for (int64_t r = 0; r < R; ++r)
+    for (int i = 0; i < 3; ++i) {
+      cp_tensor x = shard_slice(ins[i], r);
+      cp_tensor y = head_view(Y[i], qs->dtype, r, SR);
+      if ((st = cp_ulysses_permute(&x, &y, (int)U, 0, stream))) return st;
+    }
+  // 2. ring attention over the R blocks, per head group u
+  int64_t offs[CP_MAX_CHUNKS + 1];
+  if (R > CP_MAX_CHUNKS) return CP_ERR_DEGREE;
+  for (int64_t c = 0; c <= R; ++c) offs[c] = c * SR;
+  for (int64_t u = 0; u < U; ++u) {
+    cp_tensor q4, k4, v4, o4, l3;
+    cp_tensor* four[4] = {&q4, &k4, &v4, &o4};
+    uint8_t* bases[4] = {Y[0], Y[1], Y[2], Yo};
+    for (int i = 0; i < 4; ++i) {
+      const int dt = i < 3 ? qs->dtype : outs->dtype;
+      cp_tensor& t = *four[i];
+      memset(&t, 0, sizeof(t));
+      t.dtype = dt;
+      t.ndim = 4;
+      const int64_t sh[4] = {B, S, Hg, D};
+      const int64_t sd[4] = {S * Hg * D, Hg * D, D, 1};
+      for (int j = 0; j < 4; ++j) {
+        t.shape[j] = sh[j];
+        t.stride[j] = sd[j];
+      }
+      t.data = bases[i] + (size_t)(u * B * S * Hg * D) * dtype_size(dt);
+    }
+    cp_tensor* lp = nullptr;
+    if (lse) {
+      l3 = *lse;
+      l3.shape[1] = Hg;
+      l3.data = static_cast<float*>(lse->data) + u * Hg * lse->stride[1];
+      lp = &l3;
+    }
+    if ((st = ring_impl(&q4, &k4, &v4, offs, (int)R, scale, &o4, lp, stream))) return st;
+  }
+  // 3. inverse all-to-all inside every ring group r
+  for (int64_t r = 0; r < R; ++r) {
+    cp_tensor x = head_view(Yo, outs->dtype, r, SR);
+    cp_tensor y = shard_slice(outs, r);
+    if ((st = cp_ulysses_permute(&x, &y, (int)U, 1, stream))) return st;
+  }
+  return CP_OK;
+}
+
+int cp_ring_chunk_offsets(int64_t S, int R, int64_t* offsets) {
+  if (!offsets) return CP_ERR_NULL;
+  if (S < 0 || R < 1) return CP_ERR_SHAPE;
+  const int64_t c = S > 0 ? (S + R - 1) / R : 0;
+  offsets[0] = 0;
+  for (int i = 0; i < R; ++i) {
+    const int64_t nx = offsets[i] + c;
+    offsets[i + 1] = nx < S ? nx : S;
+  }
+  return CP_OK;
+}
+
+const char* cp_status_string(int status) {
+  switch (status) {
+    case CP_OK: return "ok";
+    case CP_ERR_NULL: return "null pointer or tensor";
+    case CP_ERR_DTYPE: return "unsupported or mismatched dtype";
+    case CP_ERR_SHAPE: return "bad or mismatched shape";
+    case CP_ERR_ALIGN: return "misaligned pointer or stride, or non-contiguous last dim";
+    case CP_ERR_OFFSETS: return "bad chunk offsets";
+    case CP_ERR_DEGREE: return "degree does not divide sequence length or head count";
+    case CP_ERR_CUDA: return "CUDA runtime or driver error";
+    case CP_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+    case CP_ERR_WORKSPACE: return "workspace missing or too small";
+    case CP_ERR_ALIAS: return "output overlaps an input";
+    default: return "unknown status";
+  }
+}
+
+int cp_last_device_error(void* stream) {
+  int* p = device_error_ptr();
+  if (!p) return CP_ERR_CUDA;
+  int h = 0;
+  cudaStream_t s = as_stream(stream);
+  if (cudaMemcpyAsync(&h, p, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return CP_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return CP_ERR_CUDA;
+  if (h != 0) {
+    const int zero = 0;
+    if (cudaMemcpyAsync(p, &zero, sizeof(int), cudaMemcpyHostToDevice, s) != cudaSuccess)
+      return CP_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return CP_ERR_CUDA;
+    return CP_ERR_TIMEOUT;
+  }
+  return CP_OK;
+}
+
+int cp_selftest_wait_timeout(int spin_limit, void* stream) {
+  if (spin_limit < 1 || spin_limit > (1 << 24)) return CP_ERR_SHAPE;
+  int* p = device_error_ptr();
+  if (!p) return CP_ERR_CUDA;
+  return launch_wait_timeout_selftest(spin_limit, p, as_stream(stream));
+}
+
+}  // extern "C"
+
+namespace cpattn {
+
+namespace {
+__global__ void wait_timeout_selftest_kernel(int spin_limit, int* err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // Nothing ever arrives on `bar`: the wait must give up after spin_limit
+  // polls and record the timeout.
+  if (threadIdx.x == 0) mbar_wait_polls(&bar, 0, (uint32_t)spin_limit, err);
+}
+}  // namespace
+
+int launch_wait_timeout_selftest(int spin_limit, int* dev_err, cudaStream_t stream) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(spin_limit, dev_err);
+  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+}  // namespace cpattn

@@ -1,0 +1,479 @@
+// Ring attention on the sm_100a tensor cores (bf16 in, fp32 accumulate).
+//
+// What it computes (diffusers context-parallelism guide, §Ring Attention and
+// §Ring Anything; parallelism API page, ContextParallelConfig.convert_to_fp32):
+// the local query block attends to every K/V chunk of the ring in turn; each
+// chunk's softmax statistics are folded into one fp32 accumulator at the
+// chunk boundary, which is the fp32 log-sum-exp merge of the per-chunk
+// partials.  With O kept unnormalised in tensor memory, merging the chunk
+// partial (O_c / l_c, m_c + ln l_c) into the running (O / l, m + ln l) is
+// the same rescale-and-add the online softmax does inside a chunk, so one
+// fp32 accumulator and one (m, l) pair per row carry the whole walk.  K/V
+// tiles never straddle a chunk boundary; keys past a chunk's end inside its
+// last tile are masked to -inf (that is the Ring Anything trim).
+//
+// CTA = one work unit: two 128-row query tiles of one (batch, head), so each
+// K/V tile brought in by TMA feeds four MMAs.  Warp roles (384 threads):
+//   warp 0      TMA producer: Q once, then K_j, V_j into a ring of NST slots
+//   warp 1      MMA issuer (one thread): S_t = Q_t K^T, O_t += P_t V
+//   warp 2      tensor-memory allocator
+//   warps 4-7   softmax + epilogue of query tile 0 (one row per thread)
+//   warps 8-11  softmax + epilogue of query tile 1
+// Tensor memory (512 columns x 128 lanes x 32 bit):
+//   [0,128)   S_0 (fp32), overwritten in place by P_0 (bf16, 64 columns)
+//   [128,256) S_1 / P_1
+//   [256, 256+D)  O_0;  [256+D, 256+2D)  O_1   (fp32 accumulators)
+// MMA order per key tile j (S of tile j+1 is issued as soon as P of tile j
+// has been consumed, so one softmax overlaps the other tile's MMAs):
+//   O_0 += P_0 V_j ; S_0 = Q_0 K_{j+1}^T ; O_1 += P_1 V_j ; S_1 = Q_1 K_{j+1}^T
+// tcgen05 MMAs of one CTA execute in issue order, and a commit arrives only
+// when all earlier MMAs are complete, so "S_t ready" also means the previous
+// O_t update has landed: the softmax warps may rescale O_t in place then.
+// Row statistics are per thread (one TMEM lane = one query row), so the row
+// max and row sum need no shuffles at all.
+// The softmax rescales lazily: the running max only moves when a tile's max
+// exceeds it by more than 8 (log2 units), so P <= 2^8; the final division by
+// l uses the same stale max, so the result is exact.
+
+#include <cudaTypedefs.h>
+
+#include <cstring>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace cpattn {
+
+constexpr int kTcThreads = 384;
+constexpr int kBlockM = 128;    // query rows per tile
+constexpr int kBlockN = 128;    // keys per tile
+constexpr float kRescaleThreshold = 8.0f;
+
+struct AttnTcParams {
+  CUtensorMap tmap_q;   // dims {D, S_q, H, B}, box {64, 128, 1, 1}, 128B swizzle
+  CUtensorMap tmap_k;   // dims {D, S_kv, H, B}
+  CUtensorMap tmap_v;
+  void* out;
+  float* lse;
+  int* err;
+  long long o_sb, o_ss, o_sh;    // out strides (elements)
+  long long l_sb, l_sh, l_ss;    // lse strides (elements)
+  int out_bf16;
+  int B, H, S_q, S_kv;
+  int n_q_blocks;                // ceil(S_q / 256)
+  int n_tiles;                   // key tiles over all chunks
+  int n_chunks;
+  float scale_log2;              // scale * log2(e)
+  int chunk_off[CP_MAX_CHUNKS + 1];
+};
+
+// Walks the key tiles chunk by chunk: [start, start+128) clipped to the
+// chunk end; empty chunks are skipped.
+struct TileWalk {
+  int c, start, end;
+  __device__ __forceinline__ void skip_empty(const AttnTcParams& p) {
+    while (c < p.n_chunks && p.chunk_off[c + 1] <= p.chunk_off[c]) ++c;
+    if (c < p.n_chunks) {
+      start = p.chunk_off[c];
+      end = p.chunk_off[c + 1];
+    }
+  }
+  __device__ __forceinline__ void init(const AttnTcParams& p) {
+    c = 0;
+    start = end = 0;
+    skip_empty(p);
+  }
+  __device__ __forceinline__ void next(const AttnTcParams& p) {
+    start += kBlockN;
+    if (start >= end) {
+      ++c;
+      skip_empty(p);
+    }
+  }
+  __device__ __forceinline__ int valid() const { return min(kBlockN, end - start); }
+};
+
+template <int D>
+struct TcSmem {
+  static constexpr int kTileBytes = 128 * D * 2;   // 128 rows x D bf16
+  static constexpr int kHalfBytes = 128 * 64 * 2;  // one 64-column TMA box
+};
+
+template <int D, int NST>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    attn_ring_tc_kernel(const __grid_constant__ AttnTcParams p) {
+  using L = TcSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;                                  // 2 tiles
+  uint8_t* sKV = smem + 2 * L::kTileBytes;             // NST slots
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NST * L::kTileBytes);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + NST;
+  uint64_t* s_ready = kv_empty + NST;   // [2]
+  uint64_t* p_ready = s_ready + 2;      // [2]
+  uint64_t* o_done = p_ready + 2;       // [2]
+  uint64_t* drain = o_done + 2;         // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int unit = blockIdx.x;
+  const int qblk = unit % p.n_q_blocks;
+  const int hb = unit / p.n_q_blocks;
+  const int h = hb % p.H;
+  const int b = hb / p.H;
+  const int q0 = qblk * 2 * kBlockM;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < NST; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_ready[t], 1);
+      mbar_init(&p_ready[t], kBlockM);
+      mbar_init(&o_done[t], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tmap_q);
+      tma_prefetch_desc(&p.tmap_k);
+      tma_prefetch_desc(&p.tmap_v);
+      mbar_arrive_expect_tx(q_full, 2 * L::kTileBytes);
+      for (int t = 0; t < 2; ++t)
+        for (int hh = 0; hh < D / 64; ++hh)
+          tma_load_4d(sQ + t * L::kTileBytes + hh * L::kHalfBytes, &p.tmap_q, q_full, hh * 64,
+                      q0 + t * kBlockM, h, b);
+      int last_use[NST];
+      for (int i = 0; i < NST; ++i) last_use[i] = -1;
+      TileWalk w;
+      w.init(p);
+      bool ok = true;
+      for (int n = 0; n < 2 * p.n_tiles; ++n) {
+        const int slot = n % NST;
+        const int use = n / NST;
+        if (use > 0 && !mbar_wait(&kv_empty[slot], (use - 1) & 1, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&kv_full[slot], L::kTileBytes);
+        const CUtensorMap* m = (n & 1) ? &p.tmap_v : &p.tmap_k;
+        for (int hh = 0; hh < D / 64; ++hh)
+          tma_load_4d(sKV + slot * L::kTileBytes + hh * L::kHalfBytes, m, &kv_full[slot],
+                      hh * 64, w.start, h, b);
+        last_use[slot] = use;
+        if (n & 1) w.next(p);
+      }
+      // Let every copy this CTA started land before its shared memory goes.
+      mbar_wait_drain(q_full, 0, p.err);
+      if (!ok)
+        for (int i = 0; i < NST; ++i)
+          if (last_use[i] >= 0) mbar_wait_drain(&kv_full[i], last_use[i] & 1, p.err);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, D, true);
+      const uint32_t sQa = smem_u32(sQ);
+      const uint32_t sKVa = smem_u32(sKV);
+      const uint32_t tS[2] = {tmem + 0, tmem + 128};
+      const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+
+      auto issue_s = [&](int t, int slot) {
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * L::kHalfBytes + (k & 3) * 32;
+          const uint64_t ad = smem_desc_sw128(sQa + t * L::kTileBytes + off, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(sKVa + slot * L::kTileBytes + off, 16, 1024);
+          mma_bf16_ss(tS[t], ad, bd, idesc_qk, k > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int slot, bool acc) {
+#pragma unroll
+        for (int k = 0; k < kBlockN / 16; ++k) {
+          const uint64_t bd =
+              smem_desc_sw128(sKVa + slot * L::kTileBytes + k * 2048, L::kHalfBytes, 1024);
+          mma_bf16_ts(tO[t], tS[t] + k * 8, bd, idesc_pv, (acc || k > 0) ? 1u : 0u);
+        }
+      };
+      auto wait_kv = [&](int n) -> bool {
+        if (!mbar_wait(&kv_full[n % NST], (n / NST) & 1, abort_flag, p.err)) return false;
+        tc_fence_after();
+        return true;
+      };
+
+      bool ok = mbar_wait(q_full, 0, abort_flag, p.err) && wait_kv(0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        mma_commit(&s_ready[0]);
+        issue_s(1, 0);
+        mma_commit(&s_ready[1]);
+        mma_commit(&kv_empty[0]);
+      }
+      for (int j = 0; ok && j < p.n_tiles; ++j) {
+        const int nv = 2 * j + 1, nk = 2 * j + 2;
+        const bool more = j + 1 < p.n_tiles;
+        if (!(ok = wait_kv(nv))) break;
+        if (!(ok = mbar_wait(&p_ready[0], j & 1, abort_flag, p.err))) break;
+        tc_fence_after();
+        issue_pv(0, nv % NST, j > 0);
+        if (more) {
+          if (!(ok = wait_kv(nk))) break;
+          issue_s(0, nk % NST);
+          mma_commit(&s_ready[0]);
+        } else {
+          mma_commit(&o_done[0]);
+        }
+        if (!(ok = mbar_wait(&p_ready[1], j & 1, abort_flag, p.err))) break;
+        tc_fence_after();
+        issue_pv(1, nv % NST, j > 0);
+        mma_commit(&kv_empty[nv % NST]);
+        if (more) {
+          issue_s(1, nk % NST);
+          mma_commit(&s_ready[1]);
+          mma_commit(&kv_empty[nk % NST]);
+        } else {
+          mma_commit(&o_done[1]);
+        }
+      }
+      // Every MMA issued so far must finish before tensor memory is freed.
+      mma_commit(drain);
+      mbar_wait_drain(drain, 0, p.err);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax
+    const int t = (warp - 4) >> 2;                 // query tile 0 or 1
+    const int quarter = warp & 3;                  // TMEM lane quarter
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_base + t * 128;
+    const uint32_t tO = tmem + lane_base + 256 + t * D;
+    const float sl2 = p.scale_log2;
+
+    float m_run = -INFINITY;   // running max, log2 units (scaled)
+    float l_run = 0.f;         // running sum of 2^(s*sl2 - m_run)
+    bool ok = true;
+    TileWalk w;
+    w.init(p);
+    for (int j = 0; j < p.n_tiles; ++j) {
+      if (!(ok = mbar_wait(&s_ready[t], j & 1, abort_flag, p.err))) break;
+      tc_fence_after();
+      float s[kBlockN];
+#pragma unroll
+      for (int c = 0; c < kBlockN / 32; ++c) tmem_ld32(tS + c * 32, s + c * 32);
+      tmem_wait_ld();
+      const int valid = w.valid();
+      if (valid < kBlockN) {
+#pragma unroll
+        for (int c = 0; c < kBlockN; ++c)
+          if (c >= valid) s[c] = -INFINITY;
+      }
+      float mx[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+      for (int c = 4; c < kBlockN; c += 4) {
+        mx[0] = fmaxf(mx[0], s[c]);
+        mx[1] = fmaxf(mx[1], s[c + 1]);
+        mx[2] = fmaxf(mx[2], s[c + 2]);
+        mx[3] = fmaxf(mx[3], s[c + 3]);
+      }
+      const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+      const bool need = m_tile > m_run + kRescaleThreshold;
+      if (__any_sync(0xffffffffu, need)) {
+        const float alpha = need ? ex2_approx(m_run - m_tile) : 1.0f;
+        if (need) {
+          l_run *= alpha;
+          m_run = m_tile;
+        }
+        if (j > 0) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            float o[32];
+            tmem_ld32(tO + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(tO + c * 32, o);
+          }
+        }
+      }
+      const float nm = -m_run;
+      float ls[2] = {0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < kBlockN / 32; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2_approx(fmaf(s[c * 32 + 2 * i], sl2, nm));
+          const float p1 = ex2_approx(fmaf(s[c * 32 + 2 * i + 1], sl2, nm));
+          ls[0] += p0;
+          ls[1] += p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tS + c * 16, pk);
+      }
+      l_run += ls[0] + ls[1];
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_ready[t]);
+      w.next(p);
+    }
+    if (ok && mbar_wait(&o_done[t], 0, abort_flag, p.err)) {
+      tc_fence_after();
+      const int s_row = q0 + t * kBlockM + row;
+      const bool in_range = s_row < p.S_q;
+      const float inv_l = 1.0f / l_run;
+      if (p.lse != nullptr && in_range)
+        p.lse[b * p.l_sb + h * p.l_sh + (long long)s_row * p.l_ss] =
+            (m_run + log2f(l_run)) * 0.69314718055994530942f;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        float o[32];
+        tmem_ld32(tO + c * 32, o);
+        tmem_wait_ld();
+        if (in_range) {
+          const long long base = b * p.o_sb + (long long)s_row * p.o_ss + h * p.o_sh + c * 32;
+          if (p.out_bf16) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + base);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint4 v;
+              v.x = pack_bf16x2(o[8 * i + 0] * inv_l, o[8 * i + 1] * inv_l);
+              v.y = pack_bf16x2(o[8 * i + 2] * inv_l, o[8 * i + 3] * inv_l);
+              v.z = pack_bf16x2(o[8 * i + 4] * inv_l, o[8 * i + 5] * inv_l);
+              v.w = pack_bf16x2(o[8 * i + 6] * inv_l, o[8 * i + 7] * inv_l);
+              dst[i] = v;
+            }
+          } else {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + base);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(o[4 * i] * inv_l, o[4 * i + 1] * inv_l, o[4 * i + 2] * inv_l,
+                                   o[4 * i + 3] * inv_l);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// BSHD bf16 tensor -> 4-D map {D, S, H, B}, box {64, 128, 1, 1}, 128B swizzle.
+int encode_bshd(CUtensorMap* map, const TensorView& t) {
+  auto fn = get_encode_fn();
+  if (!fn) return CP_ERR_CUDA;
+  const cuuint64_t dims[4] = {(cuuint64_t)t.shape[3], (cuuint64_t)t.shape[1],
+                              (cuuint64_t)t.shape[2], (cuuint64_t)t.shape[0]};
+  const cuuint64_t strides[3] = {(cuuint64_t)t.stride[1] * 2, (cuuint64_t)t.stride[2] * 2,
+                                 (cuuint64_t)t.stride[0] * 2};
+  const cuuint32_t box[4] = {64, 128, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t.data, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CP_OK : CP_ERR_CUDA;
+}
+
+template <int D, int NST>
+int launch_tc(const AttnTcParams& prm, int grid, cudaStream_t stream) {
+  constexpr size_t smem = 1024 + (2 + NST) * (size_t)TcSmem<D>::kTileBytes + 256;
+  auto kern = attn_ring_tc_kernel<D, NST>;
+  static bool configured[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CP_ERR_CUDA;
+  if (!configured[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return CP_ERR_CUDA;
+    configured[dev] = true;
+  }
+  kern<<<grid, kTcThreads, smem, stream>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_attn_ring_tc(const RingArgs& a, cudaStream_t stream) {
+  AttnTcParams prm;
+  memset(&prm, 0, sizeof(prm));
+  int st;
+  if ((st = encode_bshd(&prm.tmap_q, a.q)) != CP_OK) return st;
+  if ((st = encode_bshd(&prm.tmap_k, a.k)) != CP_OK) return st;
+  if ((st = encode_bshd(&prm.tmap_v, a.v)) != CP_OK) return st;
+  prm.out = a.out.data;
+  prm.out_bf16 = a.out.dtype == CP_BF16;
+  prm.o_sb = a.out.stride[0];
+  prm.o_ss = a.out.stride[1];
+  prm.o_sh = a.out.stride[2];
+  prm.lse = static_cast<float*>(a.lse.data);
+  prm.l_sb = a.lse.stride[0];
+  prm.l_sh = a.lse.stride[1];
+  prm.l_ss = a.lse.stride[2];
+  prm.err = a.dev_err;
+  prm.B = (int)a.q.shape[0];
+  prm.S_q = (int)a.q.shape[1];
+  prm.H = (int)a.q.shape[2];
+  prm.S_kv = (int)a.k.shape[1];
+  prm.n_q_blocks = (prm.S_q + 2 * kBlockM - 1) / (2 * kBlockM);
+  prm.n_chunks = a.n_chunks;
+  int n_tiles = 0;
+  for (int c = 0; c <= a.n_chunks; ++c) prm.chunk_off[c] = (int)a.chunk_off[c];
+  for (int c = 0; c < a.n_chunks; ++c) {
+    const int len = (int)(a.chunk_off[c + 1] - a.chunk_off[c]);
+    n_tiles += (len + kBlockN - 1) / kBlockN;
+  }
+  prm.n_tiles = n_tiles;
+  prm.scale_log2 = a.scale * 1.4426950408889634f;
+  const long long grid = (long long)prm.n_q_blocks * prm.H * prm.B;
+  if (grid <= 0 || n_tiles <= 0) return CP_OK;
+  if (grid > 0x7fffffffLL) return CP_ERR_SHAPE;
+  const int D = (int)a.q.shape[3];
+  if (D == 128) return launch_tc<128, 3>(prm, (int)grid, stream);
+  if (D == 64) return launch_tc<64, 4>(prm, (int)grid, stream);
+  return CP_ERR_SHAPE;
+}
+
+}  // namespace cpattn

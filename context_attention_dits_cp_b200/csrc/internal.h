@@ -1,0 +1,55 @@
+// Host-side glue shared by the C-ABI (api.cu) and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "cpattn.h"
+
+namespace cpattn {
+
+// A validated tensor: pointer, dtype and up to 6 sizes/strides in elements.
+struct TensorView {
+  void* data = nullptr;
+  int dtype = CP_F32;
+  int ndim = 0;
+  int64_t shape[CP_MAX_DIMS] = {0, 0, 0, 0, 0, 0};
+  int64_t stride[CP_MAX_DIMS] = {0, 0, 0, 0, 0, 0};
+};
+
+inline TensorView view_of(const cp_tensor* t) {
+  TensorView v;
+  if (!t) return v;
+  v.data = t->data;
+  v.dtype = t->dtype;
+  v.ndim = t->ndim;
+  for (int i = 0; i < CP_MAX_DIMS; ++i) {
+    v.shape[i] = t->shape[i];
+    v.stride[i] = t->stride[i];
+  }
+  return v;
+}
+
+inline int dtype_size(int dt) { return dt == CP_BF16 ? 2 : 4; }
+
+// Attention over a chunk list (one chunk = cp_attn_partial).
+struct RingArgs {
+  TensorView q, k, v;      // [B, S, H, D]
+  TensorView out;          // [B, S_q, H, D] f32 or bf16
+  TensorView lse;          // [B, H, S_q] f32; data may be null
+  const int64_t* chunk_off = nullptr;   // host, n_chunks + 1
+  int n_chunks = 0;
+  float scale = 0.f;
+  int* dev_err = nullptr;
+};
+
+int launch_attn_ring_tc(const RingArgs& a, cudaStream_t stream);    // bf16, tensor cores
+int launch_attn_ring_f32(const RingArgs& a, cudaStream_t stream);   // f32, FFMA
+int launch_fill_empty(const TensorView& out, const TensorView& lse, cudaStream_t stream);
+int launch_lse_merge(const TensorView& out_acc, const TensorView& lse_acc,
+                     const TensorView& out_i, const TensorView& lse_i, cudaStream_t stream);
+int launch_ulysses_permute(const TensorView& x, const TensorView& y, int degree, int dir,
+                           cudaStream_t stream);
+int launch_wait_timeout_selftest(int spin_limit, int* dev_err, cudaStream_t stream);
+
+}  // namespace cpattn

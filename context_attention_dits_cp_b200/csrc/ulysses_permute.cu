@@ -1,0 +1,136 @@
+// The Ulysses all-to-all as an on-GPU layout permutation.
+//
+// diffusers context-parallelism guide, §Ulysses Attention: the first
+// all-to-all regroups the data so that every GPU holds every token of a
+// subset of the heads; the second regroups the result by token.  With the
+// U ranks' shards held rank-major in one tensor:
+//   dir 0:  x [U, B, S/U, H, D]  ->  y [U, B, S, H/U, D]
+//           y[q, b, p*S/U + s, h', d] = x[p, b, s, q*H/U + h', d]
+//   dir 1:  the inverse, x [U, B, S, H/U, D] -> y [U, B, S/U, H, D].
+//
+// For every (destination rank, batch, token) the H/U heads of one group are
+// one contiguous run of (H/U)*D elements on both sides (1536 bytes for
+// 6 heads of 128 bf16), so the permutation is a gather of contiguous runs:
+// pure HBM traffic, one read and one write of every byte.  A warp owns one
+// run at a time (index arithmetic once per run) and moves it with 16-byte
+// vector loads, all issued before the stores; runs are walked in
+// destination order so consecutive warps write consecutive memory.
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace cpattn {
+
+namespace {
+
+struct PermParams {
+  const uint8_t* x;
+  uint8_t* y;
+  long long xs[4];   // byte strides of x dims 0..3
+  long long ys[4];   // byte strides of y dims 0..3
+  long long n_runs;
+  int U, B, Sl, Hg;
+  int run_words;     // run length in vector words
+  int dir;
+};
+
+template <typename W>
+__global__ void __launch_bounds__(256) ulysses_permute_kernel(const __grid_constant__ PermParams p) {
+  constexpr int K = 4;   // words in flight per lane
+  const int lane = threadIdx.x & 31;
+  const long long warp0 = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
+  const long long n_warps = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long r = warp0; r < p.n_runs; r += n_warps) {
+    const uint8_t* src;
+    uint8_t* dst;
+    if (p.dir == 0) {
+      // r = ((q*B + b)*U + p)*Sl + s
+      long long t = r;
+      const int s = (int)(t % p.Sl); t /= p.Sl;
+      const int pp = (int)(t % p.U); t /= p.U;
+      const int b = (int)(t % p.B);
+      const int q = (int)(t / p.B);
+      src = p.x + pp * p.xs[0] + b * p.xs[1] + s * p.xs[2] + (long long)q * p.Hg * p.xs[3];
+      dst = p.y + q * p.ys[0] + b * p.ys[1] + ((long long)pp * p.Sl + s) * p.ys[2];
+    } else {
+      // r = ((p*B + b)*Sl + s)*U + q
+      long long t = r;
+      const int q = (int)(t % p.U); t /= p.U;
+      const int s = (int)(t % p.Sl); t /= p.Sl;
+      const int b = (int)(t % p.B);
+      const int pp = (int)(t / p.B);
+      src = p.x + q * p.xs[0] + b * p.xs[1] + ((long long)pp * p.Sl + s) * p.xs[2];
+      dst = p.y + pp * p.ys[0] + b * p.ys[1] + s * p.ys[2] + (long long)q * p.Hg * p.ys[3];
+    }
+    const W* sw = reinterpret_cast<const W*>(src);
+    W* dw = reinterpret_cast<W*>(dst);
+    for (int w0 = lane; w0 < p.run_words; w0 += 32 * K) {
+      W buf[K];
+#pragma unroll
+      for (int k = 0; k < K; ++k)
+        if (w0 + 32 * k < p.run_words) buf[k] = sw[w0 + 32 * k];
+#pragma unroll
+      for (int k = 0; k < K; ++k)
+        if (w0 + 32 * k < p.run_words) dw[w0 + 32 * k] = buf[k];
+    }
+  }
+}
+
+bool aligned_to(uintptr_t v, int a) { return (v % (uintptr_t)a) == 0; }
+
+}  // namespace
+
+// x, y as validated by the C-ABI: 5-D, same dtype, (heads, D) packed.
+int launch_ulysses_permute(const TensorView& x, const TensorView& y, int U, int dir,
+                           cudaStream_t stream) {
+  const int es = dtype_size(x.dtype);
+  PermParams p;
+  p.x = static_cast<const uint8_t*>(x.data);
+  p.y = static_cast<uint8_t*>(y.data);
+  for (int i = 0; i < 4; ++i) {
+    p.xs[i] = x.stride[i] * es;
+    p.ys[i] = y.stride[i] * es;
+  }
+  p.U = U;
+  p.dir = dir;
+  p.B = (int)x.shape[1];
+  const int64_t D = x.shape[4];
+  if (dir == 0) {
+    p.Sl = (int)x.shape[2];
+    p.Hg = (int)(x.shape[3] / U);
+  } else {
+    p.Sl = (int)(x.shape[2] / U);
+    p.Hg = (int)x.shape[3];
+  }
+  // the run's head offset is taken along dim 3 of whichever side holds all H
+  // heads; its stride is D elements there.
+  const long long run_bytes = (long long)p.Hg * D * es;
+  p.n_runs = (long long)U * U * p.B * p.Sl;
+  if (p.n_runs == 0 || run_bytes == 0) return CP_OK;
+
+  int wb = 16;
+  auto ok = [&](int a) {
+    if (run_bytes % a) return false;
+    if (!aligned_to((uintptr_t)x.data, a) || !aligned_to((uintptr_t)y.data, a)) return false;
+    for (int i = 0; i < 4; ++i)
+      if (p.xs[i] % a || p.ys[i] % a) return false;
+    return true;
+  };
+  while (wb > es && !ok(wb)) wb >>= 1;
+  if (!ok(wb)) return CP_ERR_ALIGN;
+  p.run_words = (int)(run_bytes / wb);
+
+  const long long warps_needed = p.n_runs;
+  long long blocks = (warps_needed + 7) / 8;
+  const long long cap = 148LL * 8;   // 8 blocks of 256 threads per SM
+  if (blocks > cap) blocks = cap;
+  switch (wb) {
+    case 16: ulysses_permute_kernel<uint4><<<(int)blocks, 256, 0, stream>>>(p); break;
+    case 8: ulysses_permute_kernel<uint2><<<(int)blocks, 256, 0, stream>>>(p); break;
+    case 4: ulysses_permute_kernel<uint32_t><<<(int)blocks, 256, 0, stream>>>(p); break;
+    default: ulysses_permute_kernel<uint16_t><<<(int)blocks, 256, 0, stream>>>(p); break;
+  }
+  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+}  // namespace cpattn

@@ -1,0 +1,288 @@
+"""Parity of the CUDA path (through the C-ABI) with the CPU fp64 oracle.
+
+Tolerances: fp32 inputs, max-abs 1e-4 on out and lse; bf16 inputs, max-abs
+2e-2 on out and 1e-3 on lse; the Ulysses permutation is compared bit for bit.
+Small cases span several 128-row tiles with ragged tails; the five full-size
+workloads run in the same launch configuration the benchmark times and are
+checked on seeded samples of query rows the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import context_attention_dits_cp_b200 as cp
+from context_attention_dits_cp_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.float32: (1e-4, 1e-4), torch.bfloat16: (2e-2, 1e-3)}
+
+
+def _np(t):
+    return t.detach().cpu().float().numpy().astype(np.float64)
+
+
+def _dev(*ts):
+    return [t.cuda() for t in ts]
+
+
+def _check(out, lse, ref_out, ref_lse, dtype, rows=None):
+    tol_o, tol_l = TOL[dtype]
+    o = _np(out)
+    lz = _np(lse)
+    if rows is not None:
+        o = o[:, rows]
+        lz = lz[:, :, rows]
+    assert np.isfinite(o).all() and np.isfinite(lz).all()
+    eo = np.abs(o - ref_out).max()
+    el = np.abs(lz - ref_lse).max()
+    assert eo <= tol_o, f"out max-abs {eo:.3e} > {tol_o}"
+    assert el <= tol_l, f"lse max-abs {el:.3e} > {tol_l}"
+    return eo, el
+
+
+def _rows(S, n, seed):
+    rng = np.random.default_rng(seed)
+    base = np.unique(np.concatenate([[0, S - 1], rng.choice(S, size=min(n, S), replace=False)]))
+    return np.sort(base)
+
+
+# ---------------------------------------------------------------- Ulysses permute
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("U,B,S,H,D", [(2, 1, 8, 4, 64), (4, 2, 64, 8, 128), (3, 1, 30, 6, 64)])
+def test_ulysses_permute_bit_exact(cuda_ok, dtype, U, B, S, H, D):
+    x = torch.randn(U, B, S // U, H, D).to(dtype)
+    y = cp.ulysses_permute(x.cuda(), U, cp.SEQ_TO_HEAD)
+    torch.cuda.synchronize()
+    bits = lambda t: t.cpu().view(torch.int16 if dtype == torch.bfloat16 else torch.int32).numpy()
+    assert np.array_equal(bits(y), oracle.ulysses_permute(bits(x), U, 0))
+    x2 = cp.ulysses_permute(y, U, cp.HEAD_TO_SEQ)
+    assert np.array_equal(bits(x2), bits(x))
+
+
+def test_ulysses_permute_full_size_roundtrip(cuda_ok):
+    w = wl.workload("ulysses4_unified2x2")
+    q, _, _ = wl.make_workload_inputs(w)
+    x = wl.sequence_shards(q, 4)
+    y = cp.ulysses_permute(x.cuda(), 4, cp.SEQ_TO_HEAD)
+    bits = lambda t: t.cpu().view(torch.int16).numpy()
+    assert np.array_equal(bits(y), oracle.ulysses_permute(bits(x), 4, 0))
+    x2 = cp.ulysses_permute(y, 4, cp.HEAD_TO_SEQ)
+    assert torch.equal(x2.cpu().view(torch.int16), x.view(torch.int16))
+
+
+def test_ulysses_permute_into_strided_view(cuda_ok):
+    U, B, S, H, D = 2, 2, 16, 4, 64
+    x = torch.randn(U, B, S // U, H, D).to(torch.bfloat16).cuda()
+    big = torch.zeros(U, B, 2 * S, H // U, D, dtype=torch.bfloat16, device="cuda")
+    view = big[:, :, S:]
+    cp.ulysses_permute(x, U, cp.SEQ_TO_HEAD, y=view)
+    bits = lambda t: t.cpu().view(torch.int16).numpy()
+    assert np.array_equal(bits(view), oracle.ulysses_permute(bits(x), U, 0))
+    assert torch.count_nonzero(big[:, :, :S]).item() == 0
+
+
+# ---------------------------------------------------------------- LSE merge
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("in_dtype", [torch.float32, torch.bfloat16])
+def test_lse_merge(cuda_ok, D, in_dtype):
+    B, S, H = 2, 77, 3
+    g = torch.Generator().manual_seed(5)
+    oa = torch.randn(B, S, H, D, generator=g)
+    la = torch.randn(B, H, S, generator=g) * 3
+    oi = torch.randn(B, S, H, D, generator=g).to(in_dtype)
+    li = torch.randn(B, H, S, generator=g) * 3
+    # identity rows: empty partial on either side, and both empty
+    la[0, 0, :5] = -float("inf")
+    oa[0, :5, 0] = 0
+    li[1, 2, 10:15] = -float("inf")
+    la[1, 1, 20:23] = -float("inf")
+    li[1, 1, 20:23] = -float("inf")
+    oa[1, 20:23, 1] = 0
+    ref_o, ref_l = oracle.lse_merge(_np(oa), _np(la), _np(oi), _np(li))
+    da, dla = oa.cuda(), la.cuda()
+    cp.lse_merge(da, dla, oi.cuda(), li.cuda())
+    torch.cuda.synchronize()
+    assert np.abs(_np(da) - ref_o).max() <= 1e-5
+    lz = _np(dla)
+    fin = np.isfinite(ref_l)
+    assert np.array_equal(np.isneginf(lz), np.isneginf(ref_l))
+    assert np.abs(lz[fin] - ref_l[fin]).max() <= 1e-5
+
+
+# ---------------------------------------------------------------- attention, small
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("Sq,Skv", [(1, 1), (37, 200), (300, 333), (513, 129)])
+def test_attn_partial_fp32(cuda_ok, D, Sq, Skv):
+    q, k, v = wl.make_qkv(2, 3, Sq, D, torch.float32, 11, S_kv=Skv)
+    ro, rl = oracle.attention_partial(_np(q), _np(k), _np(v))
+    out, lse = cp.attn_partial(*_dev(q, k, v))
+    torch.cuda.synchronize()
+    _check(out, lse, ro, rl, torch.float32)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("Sq,Skv", [(1, 1), (128, 128), (256, 384), (300, 333), (700, 129),
+                                    (255, 1000)])
+def test_attn_partial_bf16(cuda_ok, D, Sq, Skv):
+    q, k, v = wl.make_qkv(1, 3, Sq, D, torch.bfloat16, 12, S_kv=Skv)
+    ro, rl = oracle.attention_partial(_np(q), _np(k), _np(v))
+    out, lse = cp.attn_partial(*_dev(q, k, v))
+    torch.cuda.synchronize()
+    _check(out, lse, ro, rl, torch.bfloat16)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_attn_partial_bf16_out_and_scale(cuda_ok, dtype):
+    q, k, v = wl.make_qkv(1, 2, 200, 128, dtype, 13, S_kv=260)
+    ro, rl = oracle.attention_partial(_np(q), _np(k), _np(v), scale=0.3)
+    out, lse = cp.attn_partial(*_dev(q, k, v), scale=0.3, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    _check(out, lse, ro, rl, torch.bfloat16)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_partial_never_reads_past_its_chunk(cuda_ok, dtype):
+    """Ring Anything trims padded K/V: rows after the chunk hold NaN/1e30
+    and must not leak into the partial."""
+    q, k, v = wl.make_qkv(1, 2, 150, 128, dtype, 14, S_kv=300)
+    kp, vp = k.clone(), v.clone()
+    kp[:, 201:] = float("nan")
+    vp[:, 201:] = 1e30
+    ro, rl = oracle.attention_partial(_np(q), _np(k[:, :201]), _np(v[:, :201]))
+    dk, dv = kp.cuda(), vp.cuda()
+    out, lse = cp.attn_partial(q.cuda(), dk[:, :201], dv[:, :201])
+    torch.cuda.synchronize()
+    _check(out, lse, ro, rl, dtype)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_empty_chunk_is_identity(cuda_ok, dtype):
+    q, k, v = wl.make_qkv(1, 2, 40, 64, dtype, 15, S_kv=0)
+    out, lse = cp.attn_partial(*_dev(q, k, v))
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(out).item() == 0
+    assert torch.isneginf(lse).all()
+
+
+# ---------------------------------------------------------------- ring walk, small
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("offs", [[0, 128, 256, 500], [0, 100, 100, 357, 500], [0, 500],
+                                  [0, 1, 2, 3, 250, 499, 500], [0, 0, 500, 500]])
+def test_ring_uneven_chunks(cuda_ok, dtype, offs):
+    q, k, v = wl.make_qkv(1, 2, 260, 128, dtype, 16, S_kv=500)
+    ro, rl = oracle.attention(_np(q), _np(k), _np(v))
+    out, lse = cp.ring_attention(*_dev(q, k, v), offs)
+    torch.cuda.synchronize()
+    _check(out, lse, ro, rl, dtype)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_fused_ring_matches_literal_walk(cuda_ok, dtype):
+    """cp_ring_attention (fused merge) against cp_attn_partial + cp_lse_merge
+    per chunk, in two different arrival orders."""
+    q, k, v = wl.make_qkv(2, 2, 333, 64, dtype, 17, S_kv=700)
+    dq, dk, dv = _dev(q, k, v)
+    offs = wl.chunk_offsets(wl.ring_chunk_lengths(700, 3))
+    fo, fl = cp.ring_attention(dq, dk, dv, offs)
+    for order in ([0, 1, 2], [2, 0, 1]):
+        acc = torch.zeros(2, 333, 2, 64, device="cuda")
+        lacc = torch.full((2, 2, 333), -float("inf"), device="cuda")
+        for c in order:
+            oc, lc = cp.attn_partial(dq, dk[:, offs[c]:offs[c + 1]], dv[:, offs[c]:offs[c + 1]])
+            cp.lse_merge(acc, lacc, oc, lc)
+        torch.cuda.synchronize()
+        tol_o, tol_l = TOL[dtype]
+        assert (acc - fo).abs().max().item() <= tol_o
+        assert (lacc - fl).abs().max().item() <= tol_l
+
+
+def test_constant_v_and_zero_q_closed_forms(cuda_ok):
+    g = torch.Generator().manual_seed(18)
+    S = 400
+    k = torch.randn(1, S, 2, 128, generator=g).bfloat16()
+    c = torch.randn(128, generator=g).bfloat16()
+    v = c.expand(1, S, 2, 128).contiguous()
+    q = torch.randn(1, 300, 2, 128, generator=g).bfloat16()
+    out, _ = cp.ring_attention(*_dev(q, k, v), [0, 150, 400])
+    assert (out.cpu() - c.float()).abs().max().item() <= 2e-2
+    qz = torch.zeros_like(q)
+    out, lse = cp.ring_attention(*_dev(qz, k, torch.randn(1, S, 2, 128, generator=g).bfloat16()),
+                                 [0, 400])
+    assert (lse.cpu() - np.log(S)).abs().max().item() <= 1e-3
+
+
+# ---------------------------------------------------------------- full-size workloads
+def _workload_ring(name, n_rows, seed):
+    w = wl.workload(name)
+    q, k, v = wl.make_workload_inputs(w)
+    offs = wl.chunk_offsets(wl.ring_chunk_lengths(w.S, w.ring_degree))
+    out, lse = cp.ring_attention(*_dev(q, k, v), offs)
+    torch.cuda.synchronize()
+    rows = _rows(w.S, n_rows, seed)
+    ro, rl = oracle.attention(_np(q), _np(k), _np(v), rows=rows)
+    return _check(out, lse, ro, rl, w.torch_dtype, rows=rows)
+
+
+def test_workload_tiny_ring_f32_full(cuda_ok):
+    w = wl.workload("tiny_ring_f32")
+    q, k, v = wl.make_workload_inputs(w)
+    offs = wl.chunk_offsets(wl.ring_chunk_lengths(w.S, w.ring_degree))
+    assert offs == [0, 128, 256]
+    out, lse = cp.ring_attention(*_dev(q, k, v), offs)
+    torch.cuda.synchronize()
+    ro, rl = oracle.attention(_np(q), _np(k), _np(v))
+    _check(out, lse, ro, rl, torch.float32)
+
+
+def test_workload_flux_ring4_sampled(cuda_ok):
+    _workload_ring("flux_joint_ring4", 96, 1)
+
+
+def test_workload_hires_outliers_ring8_sampled(cuda_ok):
+    _workload_ring("hires_dit_ring8", 48, 2)
+
+
+def test_workload_video_ring_anything8_sampled(cuda_ok):
+    _workload_ring("video_ring_anything8", 24, 3)
+
+
+@pytest.mark.parametrize("R,U", [(1, 4), (2, 2)])
+def test_workload_ulysses_and_unified_sampled(cuda_ok, R, U):
+    w = wl.workload("ulysses4_unified2x2")
+    q, k, v = wl.make_workload_inputs(w)
+    G = R * U
+    sh = lambda t: wl.sequence_shards(t, G)
+    out, lse = cp.usp_attention(*_dev(sh(q), sh(k), sh(v)), R, U)
+    torch.cuda.synchronize()
+    # back to token order [B, S, H, D]
+    o_full = out.cpu().transpose(0, 1).reshape(w.B, w.S, w.H, w.D)
+    rows = _rows(w.S, 32, 4 + R)
+    ro, rl = oracle.attention(_np(q), _np(k), _np(v), rows=rows)
+    _check(o_full, lse.cpu(), ro, rl, torch.bfloat16, rows=rows)
+
+
+def test_unified_small_matches_oracle_usp(cuda_ok):
+    """The emulated grid against the oracle's own rank-by-rank emulation."""
+    B, S, H, D, R, U = 2, 512, 8, 128, 2, 2
+    q, k, v = wl.make_qkv(B, H, S, D, torch.bfloat16, 19)
+    sh = lambda t: wl.sequence_shards(t, R * U)
+    out, lse = cp.usp_attention(*_dev(sh(q), sh(k), sh(v)), R, U)
+    torch.cuda.synchronize()
+    ro, rl = oracle.usp_attention(_np(sh(q)), _np(sh(k)), _np(sh(v)), R, U)
+    assert np.abs(_np(out) - ro).max() <= 2e-2
+    assert np.abs(_np(lse) - rl).max() <= 1e-3
+
+
+# ---------------------------------------------------------------- failure surfacing
+def test_bounded_wait_reports_timeout(cuda_ok):
+    assert cp.last_device_error() == 0
+    st = cp.selftest_wait_timeout(4096)
+    assert cp.binding.STATUS[st] == "CP_ERR_TIMEOUT"
+    assert cp.last_device_error() == 0   # cleared
+    # the context is still usable
+    q, k, v = wl.make_qkv(1, 1, 64, 64, torch.bfloat16, 20)
+    out, _ = cp.attn_partial(*_dev(q, k, v))
+    torch.cuda.synchronize()
+    assert torch.isfinite(out).all()
