@@ -1,0 +1,447 @@
+"""Benchmark of the context-parallel attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {cuda,reference}] [--extra]
+
+One step = one fused ring-attention pass (cp_ring_attention) over the
+FLUX-shaped joint attention workload: B=1, H=24, S=4608 (4096 image + 512
+text tokens), D=128, bf16 q/k/v, ring_degree 4 (four K/V chunks of 1152),
+fp32 output and LSE.  The headline value is 4*B*H*S^2*D / time in TFLOP/s.
+In the same run the two bandwidth-bound kernels of the path are timed on
+their own: the fp32 LSE merge (FLUX shape) and the Ulysses permutation in
+both directions (B=2, S=8192, H=24, D=128, degree 4), reported in GB/s.
+
+Timing: CUDA events on the launching stream around every step, the 126 MB
+L2 flushed (a 256 MiB buffer is overwritten) between steps outside the
+events; W untimed warm-up steps; K timed steps bracketed by a barrier and a
+device synchronise; max over ranks.  N>1 runs one independent replica of
+the workload per GPU (weak scaling, no collective on the data path).
+``--impl reference`` times the CPU fp64 oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("ring-attention TFLOP/s (4·B·H·S²·D) and % of B200 BF16 peak; "
+          "merge/permute GB/s")
+WORKLOAD = "flux_joint_ring4"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_ring_tc__flux_joint_ring4.txt")
+TC_SOURCES = ("attn_tc.cu", "common.cuh")
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def _tc_source_sha():
+    h = hashlib.sha256()
+    for f in TC_SOURCES:
+        h.update(open(os.path.join(ROOT, "context_attention_dits_cp_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def _profiled_traffic():
+    """DRAM bytes per launch of the attention kernel from the committed ncu
+    summary, or None when there is none or the kernel changed since."""
+    if not os.path.exists(PROFILE_SUMMARY):
+        return None
+    vals = {}
+    for line in open(PROFILE_SUMMARY):
+        if ":" in line and not line.startswith((" ", "#", "|")):
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_sha") != _tc_source_sha():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    NAMES = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+             0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+             0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+             0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            props = torch.cuda.get_device_properties(device_index)
+            try:
+                bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.NAMES.items():
+                    if r & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- helpers
+def _dist_init(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        if world == 1 and n_gpus > 1:
+            raise SystemExit("--gpus N>1 needs torchrun with N processes")
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = dist
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local, pg
+
+
+def _barrier(pg, dev):
+    torch.cuda.synchronize(dev)
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+
+
+def _max_over_ranks(pg, x: float, dev) -> float:
+    if pg is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _time_loop(fn, steps, warmup, flush, stream):
+    """Per-step CUDA-event times (ms) of fn(), L2 flushed between steps."""
+    for _ in range(warmup):
+        flush()
+        fn()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for a, b in evs:
+        flush()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+# ---------------------------------------------------------------- CUDA arm
+def run_cuda(args):
+    import context_attention_dits_cp_b200 as cp
+    from context_attention_dits_cp_b200 import workloads as wl
+
+    rank, world, local, pg = _dist_init(args.gpus)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    stream = torch.cuda.current_stream(dev)
+    w = wl.workload(WORKLOAD)
+    # each rank an independent replica (own seed): weak scaling
+    q, k, v = wl.make_qkv(w.B, w.H, w.S, w.D, w.torch_dtype, w.seed + 1000 * rank, w.structure)
+    offs = wl.chunk_offsets(wl.ring_chunk_lengths(w.S, w.ring_degree))
+    dq, dk, dv = q.to(dev), k.to(dev), v.to(dev)
+    out = torch.empty((w.B, w.S, w.H, w.D), dtype=torch.float32, device=dev)
+    lse = torch.empty((w.B, w.H, w.S), dtype=torch.float32, device=dev)
+    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flush = lambda: flush_buf.fill_(1)
+    step = lambda: cp.ring_attention(dq, dk, dv, offs, out=out, lse=lse)
+    flops = w.flops
+
+    # ---- timed region: K steps of the whole hot path
+    for _ in range(args.warmup):
+        flush()
+        step()
+    sampler = ClockSampler(dev.index)
+    _barrier(pg, dev)
+    with sampler:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for a, b in evs:
+            flush()
+            a.record(stream)
+            step()
+            b.record(stream)
+        _barrier(pg, dev)
+    times = [a.elapsed_time(b) for a, b in evs]
+    if args.profile_run:
+        if rank == 0:
+            print(json.dumps({"profile_run": True, "ms_per_step": float(np.mean(times))}))
+        if pg is not None:
+            pg.destroy_process_group()
+        return
+    total_ms = _max_over_ranks(pg, float(sum(times)), dev)
+    ms_per_step = total_ms / args.steps
+    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    kernel_ms = float(np.mean(times))          # one launch per step
+    gpu_launches = args.steps                  # one cp_ring_attention kernel per step
+
+    # ---- end to end through the C-ABI with host buffers
+    hq, hk, hv = (t.pin_memory() for t in (q, k, v))
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        cp.ring_attention(dq, dk, dv, offs, out=out, lse=lse)
+        hout.copy_(out, non_blocking=True)
+        hlse.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 30))
+    _barrier(pg, dev)
+    e2e_times = _time_loop(e2e_step, e2e_steps, 2, lambda: None, stream)
+    e2e_ms = _max_over_ranks(pg, float(np.mean(e2e_times)), dev)
+    h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
+    d2h = out.numel() * 4 + lse.numel() * 4
+
+    peaks, peak_src = _peaks()
+    tc_peak = float(peaks["bf16_tflops"])
+    hbm_peak = float(peaks["hbm_gbs"])
+    achieved = flops / (kernel_ms * 1e-3) / 1e12
+    traffic = _profiled_traffic()
+
+    # ---- bandwidth-bound kernels, timed on their own
+    components = {}
+    n_merge = 30 if args.steps >= 30 else max(3, args.steps)
+    acc = torch.zeros_like(out)
+    lacc = torch.full_like(lse, -float("inf"))
+    oi = torch.randn(out.shape, device=dev)
+    li = torch.randn(lse.shape, device=dev)
+    t_m = _time_loop(lambda: cp.lse_merge(acc, lacc, oi, li), n_merge, 3, flush, stream)
+    merge_bytes = out.numel() * 12 + lse.numel() * 12
+    mg = merge_bytes / (np.mean(t_m) * 1e-3) / 1e9
+    components["lse_merge"] = {"shape": [w.B, w.S, w.H, w.D], "bytes": merge_bytes,
+                               "ms": float(np.mean(t_m)), "GB/s": mg,
+                               "frac_of_hbm": mg / hbm_peak}
+    u = wl.workload("ulysses4_unified2x2")
+    x = torch.randn(4, u.B, u.S // 4, u.H, u.D, device=dev).to(torch.bfloat16)
+    y = torch.empty(4, u.B, u.S, u.H // 4, u.D, device=dev, dtype=torch.bfloat16)
+    x2 = torch.empty_like(x)
+    pbytes = 2 * x.numel() * 2
+    for name, fn in (("ulysses_permute_fwd", lambda: cp.ulysses_permute(x, 4, 0, y=y)),
+                     ("ulysses_permute_inv", lambda: cp.ulysses_permute(y, 4, 1, y=x2))):
+        t_p = _time_loop(fn, n_merge, 3, flush, stream)
+        gbs = pbytes / (np.mean(t_p) * 1e-3) / 1e9
+        components[name] = {"shape": list(x.shape), "bytes": pbytes, "ms": float(np.mean(t_p)),
+                            "GB/s": gbs, "frac_of_hbm": gbs / hbm_peak}
+    del x, y, x2, oi, li, acc, lacc
+    if args.extra:
+        components.update(_extra_workloads(cp, wl, dev, stream, flush, tc_peak))
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = _cpu_baseline(q, k, v, w)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "S": w.S, "D": w.D,
+                       "ring_degree": w.ring_degree, "chunks": [offs[i + 1] - offs[i]
+                                                                for i in range(w.ring_degree)],
+                       "inputs": "N(0,1) q/k/v, key tokens scaled by U[0.5,2]",
+                       "out": "fp32 out + fp32 lse", "l2": "flushed between steps",
+                       "per_gpu": "independent replica per GPU"},
+            "pct_of_bf16_peak": 100.0 * value / (world * tc_peak),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": tc_peak,
+                         "unit": "TFLOP/s", "frac": achieved / tc_peak, "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         "kernel": "attn_ring_tc_kernel<128,3>",
+                         "algorithmic": "4*D flops per (query, key, head): 2.609e11 per launch"},
+            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": gpu_launches,
+            "clocks": sampler.summary(),
+            "components": components,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+def _extra_workloads(cp, wl, dev, stream, flush, tc_peak):
+    res = {}
+    for name in ("hires_dit_ring8", "video_ring_anything8"):
+        w = wl.workload(name)
+        q, k, v = (t.to(dev) for t in wl.make_workload_inputs(w))
+        offs = wl.chunk_offsets(wl.ring_chunk_lengths(w.S, w.ring_degree))
+        out = torch.empty((w.B, w.S, w.H, w.D), dtype=torch.float32, device=dev)
+        lse = torch.empty((w.B, w.H, w.S), dtype=torch.float32, device=dev)
+        t = _time_loop(lambda: cp.ring_attention(q, k, v, offs, out=out, lse=lse), 5, 2,
+                       flush, stream)
+        tf = w.flops / (np.mean(t) * 1e-3) / 1e12
+        res[name] = {"ms": float(np.mean(t)), "TFLOP/s": tf, "frac_of_bf16_peak": tf / tc_peak}
+        del q, k, v, out, lse
+    u = wl.workload("ulysses4_unified2x2")
+    q, k, v = wl.make_workload_inputs(u)
+    for R, U in ((1, 4), (2, 2)):
+        sh = [wl.sequence_shards(t, R * U).to(dev) for t in (q, k, v)]
+        out = torch.empty(sh[0].shape, dtype=torch.float32, device=dev)
+        ws = torch.empty(cp.usp_workspace_bytes(u.B, u.S, u.H, u.D, torch.bfloat16,
+                                                torch.float32, R, U), dtype=torch.uint8,
+                         device=dev)
+        t = _time_loop(lambda: cp.usp_attention(*sh, R, U, out=out, workspace=ws,
+                                                want_lse=False), 5, 2, flush, stream)
+        tf = u.flops / (np.mean(t) * 1e-3) / 1e12
+        res[f"usp_R{R}_U{U}"] = {"ms": float(np.mean(t)), "TFLOP/s": tf,
+                                 "frac_of_bf16_peak": tf / tc_peak}
+    return res
+
+
+# ---------------------------------------------------------------- CPU oracle
+def _cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def _cpu_baseline(q, k, v, w, heads=None):
+    """The oracle, as it stands, on the host cores (whole workload unless
+    `heads` limits it to the first few heads)."""
+    import oracle
+    f = lambda t: t.float().numpy().astype(np.float64)
+    hs = w.H if heads is None else heads
+    qn, kn, vn = f(q[:, :, :hs]), f(k[:, :, :hs]), f(v[:, :, :hs])
+    offs = [0, w.S]
+    t0 = time.perf_counter()
+    oracle.attention(qn, kn, vn)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * w.B * hs * w.S * w.S * w.D
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": _cpu_threads(),
+            "kind": "oracle", "seconds": dt,
+            "sample": f"{WORKLOAD}: all {w.S} query rows of {hs} of {w.H} heads, fp64 one-shot"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import oracle
+    from context_attention_dits_cp_b200 import workloads as wl
+    w = wl.workload(WORKLOAD)
+    q, k, v = wl.make_workload_inputs(w)
+    f = lambda t: t.float().numpy().astype(np.float64)
+    qn, kn, vn = f(q), f(k), f(v)
+    # size one step so that warm-up + timed steps stay within ~2 minutes
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    rows = 64
+    t0 = time.perf_counter()
+    oracle.attention(qn[:, :rows], kn, vn)
+    per_row = (time.perf_counter() - t0) / rows
+    rows = int(max(16, min(w.S, budget / max(per_row, 1e-9))))
+    rng = np.random.default_rng(0)
+    for _ in range(args.warmup):
+        oracle.attention(qn, kn, vn, rows=rng.choice(w.S, rows, replace=False))
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.attention(qn, kn, vn, rows=rng.choice(w.S, rows, replace=False))
+    dt = time.perf_counter() - t0
+    flops = 4.0 * w.B * w.H * rows * w.S * w.D
+    value = args.steps * flops / dt / 1e12
+    cores = _cpu_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "S": w.S, "D": w.D,
+                   "ring_degree": w.ring_degree},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{rows} random query rows x all {w.H} heads per step "
+                                   f"against all {w.S} keys, fp64"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("cuda", "reference"), default="cuda")
+    ap.add_argument("--extra", action="store_true", help="also time the other workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-run", action="store_true",
+                    help="only the warm-up and timed ring steps (for profiler captures)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_cuda(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -48,6 +48,20 @@ constexpr int kTcThreads = 384;
 constexpr int kBlockM = 128;    // query rows per tile
 constexpr int kBlockN = 128;    // keys per tile
 constexpr float kRescaleThreshold = 8.0f;
+// Of every 8 consecutive score columns of a full key tile, this many take
+// their exponential from the FMA-pipe polynomial (exp2_fma) and the rest
+// from the MUFU unit.  Measured on B200 with the current softmax (one row
+// per thread, 208 registers): 0 is fastest (FLUX shape 1027 TFLOP/s at 0,
+// 951 at 2, 895 at 3, 845 at 4), i.e. the softmax is bound by its issue
+// latency, not by the MUFU unit, so the polynomial only adds instructions.
+#ifndef CP_EXP2_FMA_PER_8
+#define CP_EXP2_FMA_PER_8 0
+#endif
+constexpr int kExp2FmaPer8 = CP_EXP2_FMA_PER_8;
+// Register split: the producer/MMA warpgroup gives registers to the two
+// softmax warpgroups (80 + 2 * 208 <= 3 * 168 per thread, the launch budget).
+constexpr int kRegsControl = 80;
+constexpr int kRegsSoftmax = 208;
 
 struct AttnTcParams {
   CUtensorMap tmap_q;   // dims {D, S_q, H, B}, box {64, 128, 1, 1}, 128B swizzle
@@ -152,7 +166,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp < 4) {
+   regs_dec<kRegsControl>();
+   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&p.tmap_q);
@@ -163,11 +179,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int hh = 0; hh < D / 64; ++hh)
           tma_load_4d(sQ + t * L::kTileBytes + hh * L::kHalfBytes, &p.tmap_q, q_full, hh * 64,
                       q0 + t * kBlockM, h, b);
-      int last_use[NST];
-      for (int i = 0; i < NST; ++i) last_use[i] = -1;
       TileWalk w;
       w.init(p);
       bool ok = true;
+      int n_issued = 0;
       for (int n = 0; n < 2 * p.n_tiles; ++n) {
         const int slot = n % NST;
         const int use = n / NST;
@@ -180,14 +195,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int hh = 0; hh < D / 64; ++hh)
           tma_load_4d(sKV + slot * L::kTileBytes + hh * L::kHalfBytes, m, &kv_full[slot],
                       hh * 64, w.start, h, b);
-        last_use[slot] = use;
+        n_issued = n + 1;
         if (n & 1) w.next(p);
       }
       // Let every copy this CTA started land before its shared memory goes.
       mbar_wait_drain(q_full, 0, p.err);
       if (!ok)
-        for (int i = 0; i < NST; ++i)
-          if (last_use[i] >= 0) mbar_wait_drain(&kv_full[i], last_use[i] & 1, p.err);
+        for (int n = n_issued - NST < 0 ? 0 : n_issued - NST; n < n_issued; ++n)
+          mbar_wait_drain(&kv_full[n % NST], (n / NST) & 1, p.err);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -196,8 +211,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, D, true);
       const uint32_t sQa = smem_u32(sQ);
       const uint32_t sKVa = smem_u32(sKV);
-      const uint32_t tS[2] = {tmem + 0, tmem + 128};
-      const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+      // S_t / P_t at columns t*128, O_t at 256 + t*D
 
       auto issue_s = [&](int t, int slot) {
 #pragma unroll
@@ -205,7 +219,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint32_t off = (k >> 2) * L::kHalfBytes + (k & 3) * 32;
           const uint64_t ad = smem_desc_sw128(sQa + t * L::kTileBytes + off, 16, 1024);
           const uint64_t bd = smem_desc_sw128(sKVa + slot * L::kTileBytes + off, 16, 1024);
-          mma_bf16_ss(tS[t], ad, bd, idesc_qk, k > 0 ? 1u : 0u);
+          mma_bf16_ss(tmem + t * 128, ad, bd, idesc_qk, k > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, int slot, bool acc) {
@@ -213,7 +227,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int k = 0; k < kBlockN / 16; ++k) {
           const uint64_t bd =
               smem_desc_sw128(sKVa + slot * L::kTileBytes + k * 2048, L::kHalfBytes, 1024);
-          mma_bf16_ts(tO[t], tS[t] + k * 8, bd, idesc_pv, (acc || k > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + 256 + t * D, tmem + t * 128 + k * 8, bd, idesc_pv,
+                      (acc || k > 0) ? 1u : 0u);
         }
       };
       auto wait_kv = [&](int n) -> bool {
@@ -261,8 +276,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mma_commit(drain);
       mbar_wait_drain(drain, 0, p.err);
     }
-  } else if (warp >= 4) {
+   }
+  } else {
     // ------------------------------------------------------------ softmax
+    regs_inc<kRegsSoftmax>();
     const int t = (warp - 4) >> 2;                 // query tile 0 or 1
     const int quarter = warp & 3;                  // TMEM lane quarter
     const int row = quarter * 32 + lane;
@@ -319,18 +336,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       const float nm = -m_run;
       float ls[2] = {0.f, 0.f};
+      if (valid == kBlockN) {
 #pragma unroll
-      for (int c = 0; c < kBlockN / 32; ++c) {
-        uint32_t pk[16];
+        for (int c = 0; c < kBlockN / 32; ++c) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2_approx(fmaf(s[c * 32 + 2 * i], sl2, nm));
-          const float p1 = ex2_approx(fmaf(s[c * 32 + 2 * i + 1], sl2, nm));
-          ls[0] += p0;
-          ls[1] += p1;
-          pk[i] = pack_bf16x2(p0, p1);
+          for (int i = 0; i < 16; ++i) {
+            const int e = c * 32 + 2 * i;
+            const float x0 = fmaf(s[e], sl2, nm), x1 = fmaf(s[e + 1], sl2, nm);
+            const float p0 = (e & 7) < kExp2FmaPer8 ? exp2_fma(x0) : ex2_approx(x0);
+            const float p1 = ((e + 1) & 7) < kExp2FmaPer8 ? exp2_fma(x1) : ex2_approx(x1);
+            ls[0] += p0;
+            ls[1] += p1;
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tS + c * 16, pk);
         }
-        tmem_st16(tS + c * 16, pk);
+      } else {
+        // a tile cut by its chunk's end: masked columns are -inf and must
+        // give exactly 0, which the MUFU exp2 does
+#pragma unroll
+        for (int c = 0; c < kBlockN / 32; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = ex2_approx(fmaf(s[c * 32 + 2 * i], sl2, nm));
+            const float p1 = ex2_approx(fmaf(s[c * 32 + 2 * i + 1], sl2, nm));
+            ls[0] += p0;
+            ls[1] += p1;
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tS + c * 16, pk);
+        }
       }
       l_run += ls[0] + ls[1];
       tmem_wait_st();
