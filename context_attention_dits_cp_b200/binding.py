@@ -29,7 +29,8 @@ STATUS = {
     -9: "CP_ERR_WORKSPACE", -10: "CP_ERR_ALIAS",
 }
 EXPORTS = ("cp_attn_partial", "cp_lse_merge", "cp_ring_attention", "cp_ulysses_permute",
-           "cp_usp_attention", "cp_usp_workspace_bytes", "cp_ring_chunk_offsets",
+           "cp_usp_attention", "cp_usp_attention_static", "cp_usp_workspace_bytes",
+           "cp_ring_chunk_offsets",
            "cp_status_string", "cp_last_device_error", "cp_selftest_wait_timeout")
 
 
@@ -64,6 +65,7 @@ def lib() -> ctypes.CDLL:
         L.cp_ring_attention.argtypes = [P, P, P, ctypes.POINTER(i64), i32, f32, P, P, vp]
         L.cp_ulysses_permute.argtypes = [P, P, i32, i32, vp]
         L.cp_usp_attention.argtypes = [P, P, P, i32, i32, f32, vp, ctypes.c_size_t, P, P, vp]
+        L.cp_usp_attention_static.argtypes = [P, P, P, i32, i32, f32, P, P, vp]
         L.cp_usp_workspace_bytes.argtypes = [i64, i64, i64, i64, i32, i32, i32, i32]
         L.cp_usp_workspace_bytes.restype = ctypes.c_size_t
         L.cp_ring_chunk_offsets.argtypes = [i64, i32, ctypes.POINTER(i64)]
@@ -197,6 +199,29 @@ def usp_attention(q_shards, k_shards, v_shards, ring_degree: int, ulysses_degree
                                   ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
                                   _ref(do), _ref(dl), _stream(q_shards.device)),
            "cp_usp_attention")
+    return out, lse
+
+
+USP_STATIC_SCRATCH_BYTES = 64 * 1024 * 1024
+
+
+def usp_attention_static(q_shards, k_shards, v_shards, ring_degree: int, ulysses_degree: int,
+                         scale=None, out=None, lse=None, out_dtype=torch.float32, want_lse=True):
+    """usp_attention without a workspace argument, for callers that cannot
+    allocate device memory (cp_usp_attention_static): the library's fixed
+    64 MiB device array serves as the workspace; larger problems are
+    rejected with CP_ERR_WORKSPACE.  Pass preallocated `out`/`lse` to make
+    the call allocate nothing at all."""
+    G, B, Sg, H, D = q_shards.shape
+    S = G * Sg
+    out = torch.empty_like(q_shards, dtype=out_dtype) if out is None else out
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q_shards.device)
+    dq, dk, dv, do, dl = desc(q_shards), desc(k_shards), desc(v_shards), desc(out), desc(lse)
+    _check(lib().cp_usp_attention_static(_ref(dq), _ref(dk), _ref(dv), int(ring_degree),
+                                         int(ulysses_degree), _scale(scale), _ref(do), _ref(dl),
+                                         _stream(q_shards.device)),
+           "cp_usp_attention_static")
     return out, lse
 
 

@@ -168,6 +168,34 @@ size_t cp_usp_workspace_bytes(int64_t B, int64_t S, int64_t H, int64_t D,
                               int ulysses_degree);
 
 /*
+ * cp_usp_attention_static -- cp_usp_attention for callers that cannot
+ * allocate device memory.  The pages have no counterpart to this call: it
+ * exists for hosts such as another engine's plugin hook, where a cudaMalloc
+ * would synchronise the device and is not allowed, or a plain-C program with
+ * no CUDA allocator of its own.  The caller still passes inputs and outputs
+ * (same arguments and results as cp_usp_attention); the workspace is a
+ * fixed device array of CP_USP_STATIC_SCRATCH_BYTES inside the library,
+ * which every GPU that loads this part of the library holds until the
+ * process exits.  The call allocates nothing.
+ *   - Sizes whose workspace (cp_usp_workspace_bytes) exceeds
+ *     CP_USP_STATIC_SCRATCH_BYTES are rejected with CP_ERR_WORKSPACE before
+ *     any GPU work.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - Every call shares the one array and it keeps the last call's contents
+ *     (all of it is rewritten before it is read, so nothing needs clearing):
+ *     calls whose GPU work overlaps -- other streams, other threads -- race.
+ */
+#define CP_USP_STATIC_SCRATCH_BYTES (64u * 1024u * 1024u)
+int cp_usp_attention_static(const cp_tensor* q_shards,
+                            const cp_tensor* k_shards,
+                            const cp_tensor* v_shards, int ring_degree,
+                            int ulysses_degree, float scale,
+                            cp_tensor* out_shards, cp_tensor* lse,
+                            void* stream);
+
+/*
  * cp_ring_chunk_offsets -- the Ring Anything split of S tokens over R ranks:
  * ceil(S/R) tokens per rank, the last ranks holding the rest (possibly
  * nothing).  Writes R+1 offsets to the HOST array `offsets`.

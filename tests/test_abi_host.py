@@ -149,3 +149,16 @@ def test_usp_workspace_and_errors():
 def test_chunk_offsets_match_generator(S, R):
     from context_attention_dits_cp_b200 import workloads as wl
     assert bd.ring_chunk_offsets(S, R) == wl.chunk_offsets(wl.ring_chunk_lengths(S, R))
+
+
+def test_static_scratch_entry_rejects_oversize_before_any_launch():
+    """cp_usp_attention_static refuses problems whose workspace exceeds its
+    fixed array, without touching the (fake) pointers or the GPU."""
+    L = bd.lib()
+    r = ctypes.byref
+    s = lambda off, dt=bd.CP_BF16: _t([4, 1, 2048, 24, 128], dt, FAKE + off)
+    q, k, v, o = s(0), s(1 << 30), s(2 << 30), s(3 << 30, bd.CP_F32)
+    need = L.cp_usp_workspace_bytes(1, 8192, 24, 128, bd.CP_BF16, bd.CP_F32, 2, 2)
+    assert need > bd.USP_STATIC_SCRATCH_BYTES
+    assert L.cp_usp_attention_static(r(q), r(k), r(v), 2, 2, 0.0, r(o), None, None) == -9
+    assert L.cp_usp_attention_static(None, r(k), r(v), 2, 2, 0.0, r(o), None, None) == -1
