@@ -48,16 +48,31 @@ constexpr int kTcThreads = 384;
 constexpr int kBlockM = 128;    // query rows per tile
 constexpr int kBlockN = 128;    // keys per tile
 constexpr float kRescaleThreshold = 8.0f;
-// Of every 8 consecutive score columns of a full key tile, this many take
-// their exponential from the FMA-pipe polynomial (exp2_fma) and the rest
-// from the MUFU unit.  Measured on B200 with the current softmax (one row
-// per thread, 208 registers): 0 is fastest (FLUX shape 1027 TFLOP/s at 0,
-// 951 at 2, 895 at 3, 845 at 4), i.e. the softmax is bound by its issue
-// latency, not by the MUFU unit, so the polynomial only adds instructions.
-#ifndef CP_EXP2_FMA_PER_8
-#define CP_EXP2_FMA_PER_8 0
+// Of every 8 consecutive column pairs of a full key tile, this many take
+// their exponentials from the FMA-pipe polynomial (exp2_fma) and the rest
+// from the MUFU unit.
+#ifndef CP_EXP2_FMA_PAIRS_PER_8
+#define CP_EXP2_FMA_PAIRS_PER_8 0
 #endif
-constexpr int kExp2FmaPer8 = CP_EXP2_FMA_PER_8;
+constexpr int kExp2FmaPairsPer8 = CP_EXP2_FMA_PAIRS_PER_8;
+// K/V ring slots (one 128-key tile of K or V each).  Each K/V tile feeds
+// two query tiles, so a slot stays busy for most of an iteration; the ring
+// must be deep enough that the next K tile is already resident when the
+// MMA warp reaches it.
+#ifndef CP_TC_STAGES_D128
+#define CP_TC_STAGES_D128 4
+#endif
+constexpr int kStagesD128 = CP_TC_STAGES_D128;   // 64 KB Q + NST x 32 KB
+constexpr int kStagesD64 = 6;                    // 32 KB Q + NST x 16 KB
+// Speculative softmax: exponentiate a full tile against the running max
+// while finding its max, and redo the tile only if some row's max moved
+// beyond the lazy-rescale threshold.  Measured: +2.5 % on the FLUX shape,
+// -9 % on the +-8-outlier workload (whose maxima move often, so whole warps
+// redo their tiles); off by default.
+#ifndef CP_SOFTMAX_SPECULATE
+#define CP_SOFTMAX_SPECULATE 0
+#endif
+constexpr bool kSpeculativeSoftmax = CP_SOFTMAX_SPECULATE != 0;
 // Register split: the producer/MMA warpgroup gives registers to the two
 // softmax warpgroups (80 + 2 * 208 <= 3 * 168 per thread, the launch budget).
 constexpr int kRegsControl = 80;
@@ -67,6 +82,7 @@ struct AttnTcParams {
   CUtensorMap tmap_q;   // dims {D, S_q, H, B}, box {64, 128, 1, 1}, 128B swizzle
   CUtensorMap tmap_k;   // dims {D, S_kv, H, B}
   CUtensorMap tmap_v;
+  CUtensorMap tmap_out; // dims {D, S_q, H, B}, box {128 bytes of columns, 128, 1, 1}, 128B swizzle
   void* out;
   float* lse;
   int* err;
@@ -150,7 +166,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_ready[t], 1);
-      mbar_init(&p_ready[t], kBlockM);
+      mbar_init(&p_ready[t], kBlockM / 32);   // one arrive per softmax warp
       mbar_init(&o_done[t], 1);
     }
     mbar_init(drain, 1);
@@ -301,114 +317,172 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int c = 0; c < kBlockN / 32; ++c) tmem_ld32(tS + c * 32, s + c * 32);
       tmem_wait_ld();
       const int valid = w.valid();
-      if (valid < kBlockN) {
-#pragma unroll
-        for (int c = 0; c < kBlockN; ++c)
-          if (c >= valid) s[c] = -INFINITY;
-      }
-      float mx[4] = {s[0], s[1], s[2], s[3]};
-#pragma unroll
-      for (int c = 4; c < kBlockN; c += 4) {
-        mx[0] = fmaxf(mx[0], s[c]);
-        mx[1] = fmaxf(mx[1], s[c + 1]);
-        mx[2] = fmaxf(mx[2], s[c + 2]);
-        mx[3] = fmaxf(mx[3], s[c + 3]);
-      }
-      const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
-      const bool need = m_tile > m_run + kRescaleThreshold;
-      if (__any_sync(0xffffffffu, need)) {
-        const float alpha = need ? ex2_approx(m_run - m_tile) : 1.0f;
-        if (need) {
-          l_run *= alpha;
-          m_run = m_tile;
-        }
-        if (j > 0) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            float o[32];
-            tmem_ld32(tO + c * 32, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st32(tO + c * 32, o);
-          }
-        }
-      }
-      const float nm = -m_run;
-      float ls[2] = {0.f, 0.f};
-      if (valid == kBlockN) {
+      bool done = false;
+      float m_tile;
+      if (kSpeculativeSoftmax && j > 0 && valid == kBlockN) {
+        // Speculative pass: exponentiate against the running max while
+        // finding the tile max; valid unless some row's max moved by more
+        // than the lazy-rescale threshold (rare after the first tiles).
+        const float2 sl2x2 = make_float2(sl2, sl2), nmx2 = make_float2(-m_run, -m_run);
+        float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int c = 0; c < kBlockN / 32; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int e = c * 32 + 2 * i;
-            const float x0 = fmaf(s[e], sl2, nm), x1 = fmaf(s[e + 1], sl2, nm);
-            const float p0 = (e & 7) < kExp2FmaPer8 ? exp2_fma(x0) : ex2_approx(x0);
-            const float p1 = ((e + 1) & 7) < kExp2FmaPer8 ? exp2_fma(x1) : ex2_approx(x1);
-            ls[0] += p0;
-            ls[1] += p1;
-            pk[i] = pack_bf16x2(p0, p1);
+            const float2 x = fma2(make_float2(s[e], s[e + 1]), sl2x2, nmx2);
+            float2 pp;
+            if ((i & 7) < kExp2FmaPairsPer8) {
+              pp.x = exp2_fma(x.x);
+              pp.y = exp2_fma(x.y);
+            } else {
+              pp.x = ex2_approx(x.x);
+              pp.y = ex2_approx(x.y);
+            }
+            acc[i & 3] = add2(acc[i & 3], pp);
+            mx[i & 3] = max3f(mx[i & 3], s[e], s[e + 1]);
+            pk[i] = pack_bf16x2(pp.x, pp.y);
           }
           tmem_st16(tS + c * 16, pk);
         }
+        m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+        if (!__any_sync(0xffffffffu, m_tile > m_run + kRescaleThreshold)) {
+          const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
+          l_run += (a01.x + a01.y) + (a23.x + a23.y);
+          done = true;
+        }
       } else {
-        // a tile cut by its chunk's end: masked columns are -inf and must
-        // give exactly 0, which the MUFU exp2 does
+        if (valid < kBlockN) {
+#pragma unroll
+          for (int c = 0; c < kBlockN; ++c)
+            if (c >= valid) s[c] = -INFINITY;
+        }
+        float mx[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+        for (int c = 4; c < kBlockN; c += 8) {
+          mx[0] = max3f(mx[0], s[c], s[c + 1]);
+          mx[1] = max3f(mx[1], s[c + 2], s[c + 3]);
+          if (c + 4 < kBlockN) {
+            mx[2] = max3f(mx[2], s[c + 4], s[c + 5]);
+            mx[3] = max3f(mx[3], s[c + 6], s[c + 7]);
+          }
+        }
+        m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+      }
+      if (!done) {
+        // Rescale the rows whose max moved beyond the threshold, then
+        // exponentiate.  Tiles cut by their chunk's end use the MUFU unit
+        // only, which maps the masked -inf columns to exactly 0.
+        const bool need = m_tile > m_run + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? ex2_approx(m_run - m_tile) : 1.0f;
+          if (need) {
+            l_run *= alpha;
+            m_run = m_tile;
+          }
+          if (j > 0) {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              float o[32];
+              tmem_ld32(tO + c * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] *= alpha;
+              tmem_st32(tO + c * 32, o);
+            }
+          }
+        }
+        const float2 sl2x2 = make_float2(sl2, sl2), nmx2 = make_float2(-m_run, -m_run);
+        float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
         for (int c = 0; c < kBlockN / 32; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float p0 = ex2_approx(fmaf(s[c * 32 + 2 * i], sl2, nm));
-            const float p1 = ex2_approx(fmaf(s[c * 32 + 2 * i + 1], sl2, nm));
-            ls[0] += p0;
-            ls[1] += p1;
-            pk[i] = pack_bf16x2(p0, p1);
+            const int e = c * 32 + 2 * i;
+            const float2 x = fma2(make_float2(s[e], s[e + 1]), sl2x2, nmx2);
+            float2 pp;
+            if (valid == kBlockN && (i & 7) < kExp2FmaPairsPer8) {
+              pp.x = exp2_fma(x.x);
+              pp.y = exp2_fma(x.y);
+            } else {
+              pp.x = ex2_approx(x.x);
+              pp.y = ex2_approx(x.y);
+            }
+            acc[i & 3] = add2(acc[i & 3], pp);
+            pk[i] = pack_bf16x2(pp.x, pp.y);
           }
           tmem_st16(tS + c * 16, pk);
         }
+        const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
+        l_run += (a01.x + a01.y) + (a23.x + a23.y);
       }
-      l_run += ls[0] + ls[1];
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_ready[t]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_ready[t]);
       w.next(p);
     }
     if (ok && mbar_wait(&o_done[t], 0, abort_flag, p.err)) {
       tc_fence_after();
+      // Epilogue: O / l goes through this tile's Q buffer (idle once o_done
+      // fired) in 128-byte swizzled boxes of 128 rows, and leaves with TMA
+      // stores; rows past S_q are clipped by the tensor map.
       const int s_row = q0 + t * kBlockM + row;
-      const bool in_range = s_row < p.S_q;
       const float inv_l = 1.0f / l_run;
-      if (p.lse != nullptr && in_range)
+      if (p.lse != nullptr && s_row < p.S_q)
         p.lse[b * p.l_sb + h * p.l_sh + (long long)s_row * p.l_ss] =
             (m_run + log2f(l_run)) * 0.69314718055994530942f;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        float o[32];
-        tmem_ld32(tO + c * 32, o);
-        tmem_wait_ld();
-        if (in_range) {
-          const long long base = b * p.o_sb + (long long)s_row * p.o_ss + h * p.o_sh + c * 32;
+      uint8_t* stage = sQ + t * L::kTileBytes;
+      const int esz = p.out_bf16 ? 2 : 4;
+      const int cols_per_box = 128 / esz;               // 32 fp32 or 64 bf16
+      const int boxes = D / cols_per_box;               // per 128-row tile
+      const int boxes_per_round = L::kTileBytes / (128 * 128);
+      const bool leader = (warp & 3) == 0 && lane == 0;
+      for (int b0 = 0; b0 < boxes; b0 += boxes_per_round) {
+        for (int bx = b0; bx < b0 + boxes_per_round; ++bx) {
+          uint8_t* box = stage + (bx - b0) * (128 * 128) + row * 128;
+          // this box holds O columns [bx * cols_per_box, (bx+1) * cols_per_box)
           if (p.out_bf16) {
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + base);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              uint4 v;
-              v.x = pack_bf16x2(o[8 * i + 0] * inv_l, o[8 * i + 1] * inv_l);
-              v.y = pack_bf16x2(o[8 * i + 2] * inv_l, o[8 * i + 3] * inv_l);
-              v.z = pack_bf16x2(o[8 * i + 4] * inv_l, o[8 * i + 5] * inv_l);
-              v.w = pack_bf16x2(o[8 * i + 6] * inv_l, o[8 * i + 7] * inv_l);
-              dst[i] = v;
+            for (int hlf = 0; hlf < 2; ++hlf) {
+              float o[32];
+              tmem_ld32(tO + bx * 64 + hlf * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                uint4 v;
+                v.x = pack_bf16x2(o[8 * k + 0] * inv_l, o[8 * k + 1] * inv_l);
+                v.y = pack_bf16x2(o[8 * k + 2] * inv_l, o[8 * k + 3] * inv_l);
+                v.z = pack_bf16x2(o[8 * k + 4] * inv_l, o[8 * k + 5] * inv_l);
+                v.w = pack_bf16x2(o[8 * k + 6] * inv_l, o[8 * k + 7] * inv_l);
+                const int chunk = hlf * 4 + k;
+                *reinterpret_cast<uint4*>(box + ((chunk ^ (row & 7)) << 4)) = v;
+              }
             }
           } else {
-            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + base);
+            float o[32];
+            tmem_ld32(tO + bx * 32, o);
+            tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(o[4 * i] * inv_l, o[4 * i + 1] * inv_l, o[4 * i + 2] * inv_l,
-                                   o[4 * i + 3] * inv_l);
+            for (int k = 0; k < 8; ++k)
+              *reinterpret_cast<float4*>(box + ((k ^ (row & 7)) << 4)) =
+                  make_float4(o[4 * k] * inv_l, o[4 * k + 1] * inv_l, o[4 * k + 2] * inv_l,
+                              o[4 * k + 3] * inv_l);
           }
         }
+        fence_proxy_async_smem();
+        named_barrier(1 + t, kBlockM);
+        if (leader) {
+          for (int bx = b0; bx < b0 + boxes_per_round; ++bx)
+            tma_store_4d(&p.tmap_out, stage + (bx - b0) * (128 * 128), bx * cols_per_box,
+                         q0 + t * kBlockM, h, b);
+          bulk_commit();
+          bulk_wait_read_all();
+        }
+        named_barrier(1 + t, kBlockM);
       }
     }
   }
@@ -454,6 +528,25 @@ int encode_bshd(CUtensorMap* map, const TensorView& t) {
   return r == CUDA_SUCCESS ? CP_OK : CP_ERR_CUDA;
 }
 
+// Output [B, S, H, D] (f32 or bf16) -> 4-D map with 128-byte, 128-row boxes.
+int encode_out(CUtensorMap* map, const TensorView& t) {
+  auto fn = get_encode_fn();
+  if (!fn) return CP_ERR_CUDA;
+  const int es = dtype_size(t.dtype);
+  const cuuint64_t dims[4] = {(cuuint64_t)t.shape[3], (cuuint64_t)t.shape[1],
+                              (cuuint64_t)t.shape[2], (cuuint64_t)t.shape[0]};
+  const cuuint64_t strides[3] = {(cuuint64_t)t.stride[1] * es, (cuuint64_t)t.stride[2] * es,
+                                 (cuuint64_t)t.stride[0] * es};
+  const cuuint32_t box[4] = {(cuuint32_t)(128 / es), 128, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, t.dtype == CP_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                          : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                  4, t.data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CP_OK : CP_ERR_CUDA;
+}
+
 template <int D, int NST>
 int launch_tc(const AttnTcParams& prm, int grid, cudaStream_t stream) {
   constexpr size_t smem = 1024 + (2 + NST) * (size_t)TcSmem<D>::kTileBytes + 256;
@@ -480,6 +573,7 @@ int launch_attn_ring_tc(const RingArgs& a, cudaStream_t stream) {
   if ((st = encode_bshd(&prm.tmap_q, a.q)) != CP_OK) return st;
   if ((st = encode_bshd(&prm.tmap_k, a.k)) != CP_OK) return st;
   if ((st = encode_bshd(&prm.tmap_v, a.v)) != CP_OK) return st;
+  if ((st = encode_out(&prm.tmap_out, a.out)) != CP_OK) return st;
   prm.out = a.out.data;
   prm.out_bf16 = a.out.dtype == CP_BF16;
   prm.o_sb = a.out.stride[0];
@@ -508,8 +602,8 @@ int launch_attn_ring_tc(const RingArgs& a, cudaStream_t stream) {
   if (grid <= 0 || n_tiles <= 0) return CP_OK;
   if (grid > 0x7fffffffLL) return CP_ERR_SHAPE;
   const int D = (int)a.q.shape[3];
-  if (D == 128) return launch_tc<128, 3>(prm, (int)grid, stream);
-  if (D == 64) return launch_tc<64, 4>(prm, (int)grid, stream);
+  if (D == 128) return launch_tc<128, kStagesD128>(prm, (int)grid, stream);
+  if (D == 64) return launch_tc<64, kStagesD64>(prm, (int)grid, stream);
   return CP_ERR_SHAPE;
 }
 
