@@ -203,6 +203,21 @@ def run_cuda(args):
     flush = lambda: flush_buf.fill_(1)
     step = lambda: cp.ring_attention(dq, dk, dv, offs, out=out, lse=lse)
     flops = w.flops
+    if args.profile_run in ("merge", "permute"):
+        if args.profile_run == "merge":
+            acc = torch.zeros_like(out)
+            lacc = torch.full_like(lse, -float("inf"))
+            oi = torch.randn(out.shape, device=dev)
+            li = torch.randn(lse.shape, device=dev)
+            fn = lambda: cp.lse_merge(acc, lacc, oi, li)
+        else:
+            u = wl.workload("ulysses4_unified2x2")
+            x = torch.randn(4, u.B, u.S // 4, u.H, u.D, device=dev).to(torch.bfloat16)
+            y = torch.empty(4, u.B, u.S, u.H // 4, u.D, device=dev, dtype=torch.bfloat16)
+            fn = lambda: cp.ulysses_permute(x, 4, 0, y=y)
+        t = _time_loop(fn, args.steps, args.warmup, flush, stream)
+        print(json.dumps({"profile_run": args.profile_run, "ms": float(np.mean(t))}))
+        return
 
     # ---- timed region: K steps of the whole hot path
     for _ in range(args.warmup):
@@ -306,7 +321,7 @@ def run_cuda(args):
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": tc_peak,
                          "unit": "TFLOP/s", "frac": achieved / tc_peak, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16_tflops (burst)",
-                         "kernel": "attn_ring_tc_kernel<128,3>",
+                         "kernel": "attn_ring_tc_kernel<128,4>",
                          "algorithmic": "4*D flops per (query, key, head): 2.609e11 per launch"},
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -432,8 +447,9 @@ def main():
     ap.add_argument("--impl", choices=("cuda", "reference"), default="cuda")
     ap.add_argument("--extra", action="store_true", help="also time the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-run", action="store_true",
-                    help="only the warm-up and timed ring steps (for profiler captures)")
+    ap.add_argument("--profile-run", nargs="?", const="ring", default=None,
+                    choices=("ring", "merge", "permute"),
+                    help="only warm-up + timed launches of one kernel (for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -47,7 +47,15 @@ namespace cpattn {
 constexpr int kTcThreads = 384;
 constexpr int kBlockM = 128;    // query rows per tile
 constexpr int kBlockN = 128;    // keys per tile
-constexpr float kRescaleThreshold = 8.0f;
+// Lazy rescaling: the running max m of a row only moves when a tile's max
+// exceeds it by more than this many log2 units, so P <= 2^threshold.  P is
+// rounded to bf16, whose relative precision does not depend on magnitude;
+// the threshold only has to keep the fp32 accumulators finite:
+// O <= S_kv * 2^threshold * max|V| and l <= S_kv * 2^threshold.
+#ifndef CP_RESCALE_LOG2_THRESHOLD
+#define CP_RESCALE_LOG2_THRESHOLD 8
+#endif
+constexpr float kRescaleThreshold = (float)CP_RESCALE_LOG2_THRESHOLD;
 // Of every 8 consecutive column pairs of a full key tile, this many take
 // their exponentials from the FMA-pipe polynomial (exp2_fma) and the rest
 // from the MUFU unit.
@@ -64,15 +72,6 @@ constexpr int kExp2FmaPairsPer8 = CP_EXP2_FMA_PAIRS_PER_8;
 #endif
 constexpr int kStagesD128 = CP_TC_STAGES_D128;   // 64 KB Q + NST x 32 KB
 constexpr int kStagesD64 = 6;                    // 32 KB Q + NST x 16 KB
-// Speculative softmax: exponentiate a full tile against the running max
-// while finding its max, and redo the tile only if some row's max moved
-// beyond the lazy-rescale threshold.  Measured: +2.5 % on the FLUX shape,
-// -9 % on the +-8-outlier workload (whose maxima move often, so whole warps
-// redo their tiles); off by default.
-#ifndef CP_SOFTMAX_SPECULATE
-#define CP_SOFTMAX_SPECULATE 0
-#endif
-constexpr bool kSpeculativeSoftmax = CP_SOFTMAX_SPECULATE != 0;
 // Register split: the producer/MMA warpgroup gives registers to the two
 // softmax warpgroups (80 + 2 * 208 <= 3 * 168 per thread, the launch budget).
 constexpr int kRegsControl = 80;
@@ -317,61 +316,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int c = 0; c < kBlockN / 32; ++c) tmem_ld32(tS + c * 32, s + c * 32);
       tmem_wait_ld();
       const int valid = w.valid();
-      bool done = false;
-      float m_tile;
-      if (kSpeculativeSoftmax && j > 0 && valid == kBlockN) {
-        // Speculative pass: exponentiate against the running max while
-        // finding the tile max; valid unless some row's max moved by more
-        // than the lazy-rescale threshold (rare after the first tiles).
-        const float2 sl2x2 = make_float2(sl2, sl2), nmx2 = make_float2(-m_run, -m_run);
-        float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (valid < kBlockN) {
 #pragma unroll
-        for (int c = 0; c < kBlockN / 32; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int e = c * 32 + 2 * i;
-            const float2 x = fma2(make_float2(s[e], s[e + 1]), sl2x2, nmx2);
-            float2 pp;
-            if ((i & 7) < kExp2FmaPairsPer8) {
-              pp.x = exp2_fma(x.x);
-              pp.y = exp2_fma(x.y);
-            } else {
-              pp.x = ex2_approx(x.x);
-              pp.y = ex2_approx(x.y);
-            }
-            acc[i & 3] = add2(acc[i & 3], pp);
-            mx[i & 3] = max3f(mx[i & 3], s[e], s[e + 1]);
-            pk[i] = pack_bf16x2(pp.x, pp.y);
-          }
-          tmem_st16(tS + c * 16, pk);
-        }
-        m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
-        if (!__any_sync(0xffffffffu, m_tile > m_run + kRescaleThreshold)) {
-          const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
-          l_run += (a01.x + a01.y) + (a23.x + a23.y);
-          done = true;
-        }
-      } else {
-        if (valid < kBlockN) {
-#pragma unroll
-          for (int c = 0; c < kBlockN; ++c)
-            if (c >= valid) s[c] = -INFINITY;
-        }
-        float mx[4] = {s[0], s[1], s[2], s[3]};
-#pragma unroll
-        for (int c = 4; c < kBlockN; c += 8) {
-          mx[0] = max3f(mx[0], s[c], s[c + 1]);
-          mx[1] = max3f(mx[1], s[c + 2], s[c + 3]);
-          if (c + 4 < kBlockN) {
-            mx[2] = max3f(mx[2], s[c + 4], s[c + 5]);
-            mx[3] = max3f(mx[3], s[c + 6], s[c + 7]);
-          }
-        }
-        m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+        for (int c = 0; c < kBlockN; ++c)
+          if (c >= valid) s[c] = -INFINITY;
       }
-      if (!done) {
+      float mx[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+      for (int c = 4; c < kBlockN; c += 8) {
+        mx[0] = max3f(mx[0], s[c], s[c + 1]);
+        mx[1] = max3f(mx[1], s[c + 2], s[c + 3]);
+        if (c + 4 < kBlockN) {
+          mx[2] = max3f(mx[2], s[c + 4], s[c + 5]);
+          mx[3] = max3f(mx[3], s[c + 6], s[c + 7]);
+        }
+      }
+      const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+      {
         // Rescale the rows whose max moved beyond the threshold, then
         // exponentiate.  Tiles cut by their chunk's end use the MUFU unit
         // only, which maps the masked -inf columns to exactly 0.

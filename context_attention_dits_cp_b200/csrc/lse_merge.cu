@@ -9,10 +9,11 @@
 //
 // HBM-bound: per output row of D floats it reads out_acc and out_i and
 // writes out_acc back (12 bytes per fp32 element, 10 with a bf16 out_i) plus
-// 12 bytes of LSE.  One warp owns 32 consecutive tokens of one (batch,
-// head): lane t reads both LSEs of token t with one coalesced 128-byte load,
-// computes the two weights, and the warp then streams the 32 output rows,
-// each lane moving D/32 consecutive elements with one vector access.
+// 12 bytes of LSE.  One warp owns 8 consecutive tokens of one (batch, head):
+// it loads their two LSEs and all 8 rows of both partials at once (one
+// memory round trip), computes the two weights per token, and writes the 8
+// merged rows, each lane moving D/32 consecutive elements per row with one
+// vector access.
 
 #include "common.cuh"
 #include "internal.h"
@@ -50,7 +51,7 @@ struct InVec {
     if constexpr (BF16_IN) {
       const __nv_bfloat16* p = reinterpret_cast<const __nv_bfloat16*>(base) + off;
       if constexpr (V == 4) {
-        const uint2 u = *reinterpret_cast<const uint2*>(p);
+        const uint2 u = __ldcs(reinterpret_cast<const uint2*>(p));
         const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
         const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
         x[0] = __low2float(a);
@@ -58,81 +59,101 @@ struct InVec {
         x[2] = __low2float(b);
         x[3] = __high2float(b);
       } else {
-        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(p);
+        const unsigned int w = __ldcs(reinterpret_cast<const unsigned int*>(p));
+        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&w);
         x[0] = __low2float(a);
         x[1] = __high2float(a);
       }
     } else {
       const float* p = reinterpret_cast<const float*>(base) + off;
       if constexpr (V == 4) {
-        const float4 u = *reinterpret_cast<const float4*>(p);
+        const float4 u = __ldcs(reinterpret_cast<const float4*>(p));
         x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
       } else {
-        const float2 u = *reinterpret_cast<const float2*>(p);
+        const float2 u = __ldcs(reinterpret_cast<const float2*>(p));
         x[0] = u.x; x[1] = u.y;
       }
     }
   }
 };
 
+// One warp owns kTok consecutive tokens of one (batch, head).  All of its
+// row loads are issued together with the two LSE loads, so a warp needs a
+// single memory round trip; loads and stores use the streaming (evict-first)
+// cache policy since every byte is touched exactly once.
+#ifndef CP_MERGE_TOKENS_PER_WARP
+#define CP_MERGE_TOKENS_PER_WARP 8
+#endif
+constexpr int kTok = CP_MERGE_TOKENS_PER_WARP;
+#ifndef CP_MERGE_BLOCKS
+#define CP_MERGE_BLOCKS (148 * 8)
+#endif
+constexpr long long kMergeBlocks = CP_MERGE_BLOCKS;
+
 template <int D, bool BF16_IN>
 __global__ void __launch_bounds__(256) lse_merge_kernel(const __grid_constant__ MergeParams p) {
   constexpr int V = D / 32;   // elements per lane per row
-  constexpr int U = 4;        // rows in flight per lane
+  using FV = typename F32Vec<V>::T;
   const int lane = threadIdx.x & 31;
-  const long long gw = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
-  const int sb = (int)(gw % p.n_sblocks);
-  const long long hb = gw / p.n_sblocks;
-  const int h = (int)(hb % p.H);
-  const int b = (int)(hb / p.H);
-  if (b >= p.B) return;
+  const long long n_groups = (long long)p.n_sblocks * p.H * p.B;
+  const long long n_warps = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long gw = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5; gw < n_groups;
+       gw += n_warps) {
+  // heads fastest: neighbouring warps merge neighbouring rows in memory
+  const int h = (int)(gw % p.H);
+  const long long sbb = gw / p.H;
+  const int sb = (int)(sbb % p.n_sblocks);
+  const int b = (int)(sbb / p.n_sblocks);
+  const int s0 = sb * kTok;
+  const int n_rows = min(kTok, p.S - s0);
 
-  const int s0 = sb * 32;
-  const int s = s0 + lane;
-  float wa = 1.f, wb = 0.f;
-  if (s < p.S) {
-    float* la_p = p.lse_acc + b * p.la_sb + h * p.la_sh + (long long)s * p.la_ss;
-    const float a = *la_p;
-    const float bb = p.lse_i[b * p.li_sb + h * p.li_sh + (long long)s * p.li_ss];
-    if (!(a == -INFINITY && bb == -INFINITY)) {
-      const float mx = fmaxf(a, bb);
-      const float nl = mx + log1pf(expf(-fabsf(a - bb)));
-      wa = expf(a - nl);
-      wb = expf(bb - nl);
-      *la_p = nl;
+  // lanes 0..kTok-1 read lse_acc, lanes 16..16+kTok-1 read lse_i
+  float lv = -INFINITY;
+  {
+    const int tk = lane & 15;
+    if (tk < n_rows) {
+      const long long s = s0 + tk;
+      lv = lane < 16 ? __ldcs(p.lse_acc + b * p.la_sb + h * p.la_sh + s * p.la_ss)
+                     : __ldcs(p.lse_i + b * p.li_sb + h * p.li_sh + s * p.li_ss);
     }
   }
-  const int n_rows = min(32, p.S - s0);
-  for (int t0 = 0; t0 < n_rows; t0 += U) {
-    float x[U][V], y[U][V], ws[U][2];
+  float x[kTok][V], y[kTok][V];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int t = t0 + u;
-      ws[u][0] = __shfl_sync(0xffffffffu, wa, t & 31);
-      ws[u][1] = __shfl_sync(0xffffffffu, wb, t & 31);
-      if (t < n_rows) {
-        const long long sr = s0 + t;
-        const float* ap = p.acc + b * p.a_sb + sr * p.a_ss + h * p.a_sh + lane * V;
-        const typename F32Vec<V>::T av = *reinterpret_cast<const typename F32Vec<V>::T*>(ap);
-        const float* af = reinterpret_cast<const float*>(&av);
+  for (int t = 0; t < kTok; ++t) {
+    if (t < n_rows) {
+      const long long sr = s0 + t;
+      const FV av = __ldcs(reinterpret_cast<const FV*>(p.acc + b * p.a_sb + sr * p.a_ss +
+                                                        h * p.a_sh + lane * V));
+      const float* af = reinterpret_cast<const float*>(&av);
 #pragma unroll
-        for (int i = 0; i < V; ++i) x[u][i] = af[i];
-        InVec<V, BF16_IN>::load(p.oi, b * p.i_sb + sr * p.i_ss + h * p.i_sh + lane * V, y[u]);
-      }
+      for (int i = 0; i < V; ++i) x[t][i] = af[i];
+      InVec<V, BF16_IN>::load(p.oi, b * p.i_sb + sr * p.i_ss + h * p.i_sh + lane * V, y[t]);
     }
+  }
+  // weights of token `lane` (lanes 0..kTok-1)
+  const float a = lv;
+  const float bb = __shfl_sync(0xffffffffu, lv, (lane & 15) + 16);
+  float wa = 1.f, wb = 0.f;
+  if (lane < n_rows && !(a == -INFINITY && bb == -INFINITY)) {
+    const float mx = fmaxf(a, bb);
+    const float nl = mx + log1pf(expf(-fabsf(a - bb)));
+    wa = expf(a - nl);
+    wb = expf(bb - nl);
+    __stcs(p.lse_acc + b * p.la_sb + h * p.la_sh + (long long)(s0 + lane) * p.la_ss, nl);
+  }
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int t = t0 + u;
-      if (t < n_rows) {
-        const long long sr = s0 + t;
-        float r[V];
+  for (int t = 0; t < kTok; ++t) {
+    const float ca = __shfl_sync(0xffffffffu, wa, t);
+    const float cb = __shfl_sync(0xffffffffu, wb, t);
+    if (t < n_rows) {
+      const long long sr = s0 + t;
+      float r[V];
 #pragma unroll
-        for (int i = 0; i < V; ++i) r[i] = ws[u][0] * x[u][i] + ws[u][1] * y[u][i];
-        float* ap = p.acc + b * p.a_sb + sr * p.a_ss + h * p.a_sh + lane * V;
-        *reinterpret_cast<typename F32Vec<V>::T*>(ap) =
-            *reinterpret_cast<const typename F32Vec<V>::T*>(r);
-      }
+      for (int i = 0; i < V; ++i) r[i] = ca * x[t][i] + cb * y[t][i];
+      __stcs(reinterpret_cast<FV*>(p.acc + b * p.a_sb + sr * p.a_ss + h * p.a_sh + lane * V),
+             *reinterpret_cast<const FV*>(r));
     }
+  }
   }
 }
 
@@ -160,12 +181,14 @@ int launch_lse_merge(const TensorView& acc, const TensorView& lse_acc, const Ten
   p.B = (int)acc.shape[0];
   p.S = (int)acc.shape[1];
   p.H = (int)acc.shape[2];
-  p.n_sblocks = (p.S + 31) / 32;
+  p.n_sblocks = (p.S + kTok - 1) / kTok;
   const int D = (int)acc.shape[3];
   const long long warps = (long long)p.n_sblocks * p.H * p.B;
   if (warps <= 0) return CP_OK;
-  const long long blocks = (warps + 7) / 8;
-  if (blocks > 0x7fffffffLL) return CP_ERR_SHAPE;
+  // persistent grid: 8 blocks of 8 warps per SM, grid-stride over the
+  // token groups, so all warps start together and finish together
+  long long blocks = (warps + 7) / 8;
+  if (blocks > kMergeBlocks) blocks = kMergeBlocks;
   const bool bf = oi.dtype == CP_BF16;
   if (D == 128 && !bf) lse_merge_kernel<128, false><<<(int)blocks, 256, 0, stream>>>(p);
   else if (D == 128 && bf) lse_merge_kernel<128, true><<<(int)blocks, 256, 0, stream>>>(p);
