@@ -154,18 +154,28 @@ def _dist_init(n_gpus):
 
 
 def _barrier(pg, dev):
-    torch.cuda.synchronize(dev)
+    """Device synchronise, then a barrier over all ranks, then synchronise."""
+    if dev.type == "cuda":
+        torch.cuda.synchronize(dev)
     if pg is not None:
         pg.barrier()
-    torch.cuda.synchronize(dev)
+    if dev.type == "cuda":
+        torch.cuda.synchronize(dev)
 
 
 def _max_over_ranks(pg, x: float, dev) -> float:
+    """The largest of every rank's `x` (the slowest rank sets the job time)."""
     if pg is None:
         return x
     t = torch.tensor([x], dtype=torch.float64, device=dev)
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world: int, flops_per_rank_step: float, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: every rank runs its own replica of the step, and
+    the job's step time is the slowest rank's."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
 
 
 def _time_loop(fn, steps, warmup, flush, stream):
@@ -243,7 +253,7 @@ def run_cuda(args):
         return
     total_ms = _max_over_ranks(pg, float(sum(times)), dev)
     ms_per_step = total_ms / args.steps
-    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    value = job_throughput(world, flops, ms_per_step)
     kernel_ms = float(np.mean(times))          # one launch per step
     gpu_launches = args.steps                  # one cp_ring_attention kernel per step
 
