@@ -81,7 +81,21 @@ float resolve_scale(float scale, int64_t D) {
   return scale;
 }
 
-int launch_status(int st) { return st; }
+// The unified composition folds its permutations into the attention
+// kernel's tensor maps (one launch, no intermediates) for bf16 inputs when
+// every 128-row tile lies inside one sequence shard.
+bool usp_fusable_sizes(int in_dtype, int64_t D, int64_t G, int64_t Sg) {
+  return in_dtype == CP_BF16 && (D == 64 || D == 128) && (G == 1 || Sg % 128 == 0);
+}
+
+// Workspace of the unfused composition: head-sharded q, k, v and output,
+// each [U, B, S, H/U, D], 256-byte aligned.
+size_t usp_unfused_bytes(int64_t B, int64_t S, int64_t H, int64_t D, int in_dtype,
+                         int out_dtype) {
+  const size_t n = (size_t)B * S * H * D;
+  auto rnd = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  return 3 * rnd(n * dtype_size(in_dtype)) + rnd(n * dtype_size(out_dtype));
+}
 
 // Shared validation of attention arguments.  On success fills `a` (without
 // chunk offsets) and reports whether there is anything to compute.
@@ -254,9 +268,9 @@ size_t cp_usp_workspace_bytes(int64_t B, int64_t S, int64_t H, int64_t D, int in
   if (B < 0 || S < 0 || H < 0 || D < 0 || ring_degree < 1 || ulysses_degree < 1) return 0;
   if ((in_dtype != CP_F32 && in_dtype != CP_BF16) || (out_dtype != CP_F32 && out_dtype != CP_BF16))
     return 0;
-  const size_t n = (size_t)B * S * H * D;   // elements of one full tensor
-  auto rnd = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  return 3 * rnd(n * dtype_size(in_dtype)) + rnd(n * dtype_size(out_dtype));
+  const int64_t G = (int64_t)ring_degree * ulysses_degree;
+  if (usp_fusable_sizes(in_dtype, D, G, G > 0 ? S / G : 0)) return 0;   // no intermediates
+  return usp_unfused_bytes(B, S, H, D, in_dtype, out_dtype);
 }
 
 int cp_usp_attention(const cp_tensor* qs, const cp_tensor* ks, const cp_tensor* vs,
@@ -283,12 +297,42 @@ int cp_usp_attention(const cp_tensor* qs, const cp_tensor* ks, const cp_tensor* 
     if (lse->dtype != CP_F32) return CP_ERR_DTYPE;
     if (lse->shape[0] != B || lse->shape[1] != H || lse->shape[2] != S) return CP_ERR_SHAPE;
   }
-  const size_t need =
-      cp_usp_workspace_bytes(B, S, H, D, qs->dtype, outs->dtype, ring_degree, ulysses_degree);
-  if (!workspace) return CP_ERR_WORKSPACE;
-  if (workspace_bytes < need) return CP_ERR_WORKSPACE;
-  if (reinterpret_cast<uintptr_t>(workspace) % 256) return CP_ERR_ALIGN;
+  if (R > CP_MAX_CHUNKS) return CP_ERR_DEGREE;
   if (B == 0 || S == 0 || H == 0) return CP_OK;
+
+  // Fused: attention reads q/k/v and writes out in the shard layout through
+  // 5-D tensor maps; head group u of ring rank r is just heads u*H/U.. of
+  // tokens r*S/R.., so one launch over all heads with R chunks is the whole
+  // grid.
+  if (usp_fusable_sizes(qs->dtype, D, G, Sg) && outs->stride[4] == 1 &&
+      check_vector_layout(qs, 16) == CP_OK && check_vector_layout(ks, 16) == CP_OK &&
+      check_vector_layout(vs, 16) == CP_OK && check_vector_layout(outs, 16) == CP_OK) {
+    RingArgs a;
+    a.q = view_of(qs);
+    a.k = view_of(ks);
+    a.v = view_of(vs);
+    a.out = view_of(outs);
+    a.lse = view_of(lse);
+    if (overlaps(a.out, a.q) || overlaps(a.out, a.k) || overlaps(a.out, a.v)) return CP_ERR_ALIAS;
+    if (lse && (overlaps(a.lse, a.q) || overlaps(a.lse, a.k) || overlaps(a.lse, a.v) ||
+                overlaps(a.lse, a.out)))
+      return CP_ERR_ALIAS;
+    int64_t foffs[CP_MAX_CHUNKS + 1];
+    for (int64_t c = 0; c <= R; ++c) foffs[c] = c * SR;
+    a.chunk_off = foffs;
+    a.n_chunks = (int)R;
+    a.scale = resolve_scale(scale, D);
+    a.dev_err = device_error_ptr();
+    if (!a.dev_err) return CP_ERR_CUDA;
+    return launch_attn_ring_tc(a, as_stream(stream));
+  }
+
+  // Unfused: Ulysses permute -> ring attention per head group -> inverse
+  // permute, through the caller's workspace.
+  if (!workspace) return CP_ERR_WORKSPACE;
+  if (workspace_bytes < usp_unfused_bytes(B, S, H, D, qs->dtype, outs->dtype))
+    return CP_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return CP_ERR_ALIGN;
 
   const size_t n = (size_t)B * S * H * D;
   auto rnd = [](size_t x) { return (x + 255) & ~(size_t)255; };
@@ -328,7 +372,6 @@ int cp_usp_attention(const cp_tensor* qs, const cp_tensor* ks, const cp_tensor* 
     }
   // 2. ring attention over the R blocks, per head group u
   int64_t offs[CP_MAX_CHUNKS + 1];
-  if (R > CP_MAX_CHUNKS) return CP_ERR_DEGREE;
   for (int64_t c = 0; c <= R; ++c) offs[c] = c * SR;
   for (int64_t u = 0; u < U; ++u) {
     cp_tensor q4, k4, v4, o4, l3;

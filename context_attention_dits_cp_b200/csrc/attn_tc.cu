@@ -78,17 +78,20 @@ constexpr int kRegsControl = 80;
 constexpr int kRegsSoftmax = 208;
 
 struct AttnTcParams {
-  CUtensorMap tmap_q;   // dims {D, S_q, H, B}, box {64, 128, 1, 1}, 128B swizzle
-  CUtensorMap tmap_k;   // dims {D, S_kv, H, B}
+  // 5-D maps {D, seg, H, G, B}: token s of the sequence is row s % seg of
+  // segment s / seg.  Plain [B, S, H, D] tensors have one segment (G = 1);
+  // Ulysses sequence shards [G, B, S/G, H, D] are read and written in place.
+  CUtensorMap tmap_q;   // box {64, 128, 1, 1, 1}, 128B swizzle
+  CUtensorMap tmap_k;
   CUtensorMap tmap_v;
-  CUtensorMap tmap_out; // dims {D, S_q, H, B}, box {128 bytes of columns, 128, 1, 1}, 128B swizzle
+  CUtensorMap tmap_out; // box {128 bytes of columns, 128, 1, 1, 1}, 128B swizzle
   void* out;
   float* lse;
   int* err;
-  long long o_sb, o_ss, o_sh;    // out strides (elements)
   long long l_sb, l_sh, l_ss;    // lse strides (elements)
   int out_bf16;
   int B, H, S_q, S_kv;
+  int seg_q, seg_kv;             // tokens per segment (S itself for one segment)
   int n_q_blocks;                // ceil(S_q / 256)
   int n_tiles;                   // key tiles over all chunks
   int n_chunks;
@@ -144,7 +147,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* s_ready = kv_empty + NST;   // [2]
   uint64_t* p_ready = s_ready + 2;      // [2]
   uint64_t* o_done = p_ready + 2;       // [2]
-  uint64_t* drain = o_done + 2;         // [1]
+  uint64_t* epi_full = o_done + 2;      // [2] a round of staged output is in smem
+  uint64_t* epi_free = epi_full + 2;    // [2] TMA has read the staged round
+  uint64_t* drain = epi_free + 2;       // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -167,6 +172,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&s_ready[t], 1);
       mbar_init(&p_ready[t], kBlockM / 32);   // one arrive per softmax warp
       mbar_init(&o_done[t], 1);
+      mbar_init(&epi_full[t], kBlockM / 32);   // one arrive per softmax warp
+      mbar_init(&epi_free[t], 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -190,10 +197,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tma_prefetch_desc(&p.tmap_k);
       tma_prefetch_desc(&p.tmap_v);
       mbar_arrive_expect_tx(q_full, 2 * L::kTileBytes);
-      for (int t = 0; t < 2; ++t)
+      for (int t = 0; t < 2; ++t) {
+        const int r0 = q0 + t * kBlockM;
         for (int hh = 0; hh < D / 64; ++hh)
-          tma_load_4d(sQ + t * L::kTileBytes + hh * L::kHalfBytes, &p.tmap_q, q_full, hh * 64,
-                      q0 + t * kBlockM, h, b);
+          tma_load_5d(sQ + t * L::kTileBytes + hh * L::kHalfBytes, &p.tmap_q, q_full, hh * 64,
+                      r0 % p.seg_q, h, r0 / p.seg_q, b);
+      }
       TileWalk w;
       w.init(p);
       bool ok = true;
@@ -208,8 +217,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mbar_arrive_expect_tx(&kv_full[slot], L::kTileBytes);
         const CUtensorMap* m = (n & 1) ? &p.tmap_v : &p.tmap_k;
         for (int hh = 0; hh < D / 64; ++hh)
-          tma_load_4d(sKV + slot * L::kTileBytes + hh * L::kHalfBytes, m, &kv_full[slot],
-                      hh * 64, w.start, h, b);
+          tma_load_5d(sKV + slot * L::kTileBytes + hh * L::kHalfBytes, m, &kv_full[slot],
+                      hh * 64, w.start % p.seg_kv, h, w.start / p.seg_kv, b);
         n_issued = n + 1;
         if (n & 1) w.next(p);
       }
@@ -386,11 +395,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lane == 0) mbar_arrive(&p_ready[t]);
       w.next(p);
     }
+    int rounds = 0;   // epilogue rounds staged (phase of epi_full / epi_free)
     if (ok && mbar_wait(&o_done[t], 0, abort_flag, p.err)) {
       tc_fence_after();
       // Epilogue: O / l goes through this tile's Q buffer (idle once o_done
       // fired) in 128-byte swizzled boxes of 128 rows, and leaves with TMA
-      // stores; rows past S_q are clipped by the tensor map.
+      // stores; rows past S_q are clipped by the tensor map.  The warps hand
+      // the staging buffer to the storing thread and back through bounded
+      // mbarrier waits, so a warp that gave up never blocks the others.
       const int s_row = q0 + t * kBlockM + row;
       const float inv_l = 1.0f / l_run;
       if (p.lse != nullptr && s_row < p.S_q)
@@ -402,7 +414,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int boxes = D / cols_per_box;               // per 128-row tile
       const int boxes_per_round = L::kTileBytes / (128 * 128);
       const bool leader = (warp & 3) == 0 && lane == 0;
-      for (int b0 = 0; b0 < boxes; b0 += boxes_per_round) {
+      for (int b0 = 0; ok && b0 < boxes; b0 += boxes_per_round, ++rounds) {
+        // the previous round's TMA stores must have read the staging buffer
+        if (rounds > 0 && !(ok = mbar_wait(&epi_free[t], (rounds - 1) & 1, abort_flag, p.err)))
+          break;
         for (int bx = b0; bx < b0 + boxes_per_round; ++bx) {
           uint8_t* box = stage + (bx - b0) * (128 * 128) + row * 128;
           // this box holds O columns [bx * cols_per_box, (bx+1) * cols_per_box)
@@ -435,17 +450,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
         fence_proxy_async_smem();
-        named_barrier(1 + t, kBlockM);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&epi_full[t]);
         if (leader) {
+          if (!(ok = mbar_wait(&epi_full[t], rounds & 1, abort_flag, p.err))) break;
+          const int r0 = q0 + t * kBlockM;
           for (int bx = b0; bx < b0 + boxes_per_round; ++bx)
-            tma_store_4d(&p.tmap_out, stage + (bx - b0) * (128 * 128), bx * cols_per_box,
-                         q0 + t * kBlockM, h, b);
+            tma_store_5d(&p.tmap_out, stage + (bx - b0) * (128 * 128), bx * cols_per_box,
+                         r0 % p.seg_q, h, r0 / p.seg_q, b);
           bulk_commit();
           bulk_wait_read_all();
+          mbar_arrive(&epi_free[t]);
         }
-        named_barrier(1 + t, kBlockM);
       }
     }
+    // shared memory must not be released while TMA still reads it
+    if (rounds > 0) mbar_wait_drain(&epi_free[t], (rounds - 1) & 1, p.err);
   }
 
   tc_fence_before();
@@ -473,36 +493,51 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-// BSHD bf16 tensor -> 4-D map {D, S, H, B}, box {64, 128, 1, 1}, 128B swizzle.
-int encode_bshd(CUtensorMap* map, const TensorView& t) {
+// The five extents/strides of a [B, S, H, D] view (one segment) or of a
+// [G, B, S/G, H, D] shard view, as {D, seg, H, G, B}; strides in bytes of
+// dims 1..4.
+void seg_geometry(const TensorView& t, cuuint64_t dims[5], cuuint64_t strides[4]) {
+  const cuuint64_t es = dtype_size(t.dtype);
+  if (t.ndim == 4) {
+    dims[0] = t.shape[3]; dims[1] = t.shape[1]; dims[2] = t.shape[2]; dims[3] = 1;
+    dims[4] = t.shape[0];
+    strides[0] = t.stride[1] * es; strides[1] = t.stride[2] * es;
+    strides[2] = t.stride[1] * es * (t.shape[1] > 0 ? t.shape[1] : 1);
+    strides[3] = t.stride[0] * es;
+  } else {
+    dims[0] = t.shape[4]; dims[1] = t.shape[2]; dims[2] = t.shape[3]; dims[3] = t.shape[0];
+    dims[4] = t.shape[1];
+    strides[0] = t.stride[2] * es; strides[1] = t.stride[3] * es; strides[2] = t.stride[0] * es;
+    strides[3] = t.stride[1] * es;
+  }
+}
+
+// bf16 q/k/v -> 5-D map, box {64, 128, 1, 1, 1}, 128B swizzle.
+int encode_in(CUtensorMap* map, const TensorView& t) {
   auto fn = get_encode_fn();
   if (!fn) return CP_ERR_CUDA;
-  const cuuint64_t dims[4] = {(cuuint64_t)t.shape[3], (cuuint64_t)t.shape[1],
-                              (cuuint64_t)t.shape[2], (cuuint64_t)t.shape[0]};
-  const cuuint64_t strides[3] = {(cuuint64_t)t.stride[1] * 2, (cuuint64_t)t.stride[2] * 2,
-                                 (cuuint64_t)t.stride[0] * 2};
-  const cuuint32_t box[4] = {64, 128, 1, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t.data, dims, strides, box, estr,
+  cuuint64_t dims[5], strides[4];
+  seg_geometry(t, dims, strides);
+  const cuuint32_t box[5] = {64, 128, 1, 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, t.data, dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? CP_OK : CP_ERR_CUDA;
 }
 
-// Output [B, S, H, D] (f32 or bf16) -> 4-D map with 128-byte, 128-row boxes.
+// Output (f32 or bf16) -> 5-D map with 128-byte, 128-row boxes.
 int encode_out(CUtensorMap* map, const TensorView& t) {
   auto fn = get_encode_fn();
   if (!fn) return CP_ERR_CUDA;
   const int es = dtype_size(t.dtype);
-  const cuuint64_t dims[4] = {(cuuint64_t)t.shape[3], (cuuint64_t)t.shape[1],
-                              (cuuint64_t)t.shape[2], (cuuint64_t)t.shape[0]};
-  const cuuint64_t strides[3] = {(cuuint64_t)t.stride[1] * es, (cuuint64_t)t.stride[2] * es,
-                                 (cuuint64_t)t.stride[0] * es};
-  const cuuint32_t box[4] = {(cuuint32_t)(128 / es), 128, 1, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  cuuint64_t dims[5], strides[4];
+  seg_geometry(t, dims, strides);
+  const cuuint32_t box[5] = {(cuuint32_t)(128 / es), 128, 1, 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = fn(map, t.dtype == CP_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                  4, t.data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  5, t.data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? CP_OK : CP_ERR_CUDA;
@@ -531,24 +566,32 @@ int launch_attn_ring_tc(const RingArgs& a, cudaStream_t stream) {
   AttnTcParams prm;
   memset(&prm, 0, sizeof(prm));
   int st;
-  if ((st = encode_bshd(&prm.tmap_q, a.q)) != CP_OK) return st;
-  if ((st = encode_bshd(&prm.tmap_k, a.k)) != CP_OK) return st;
-  if ((st = encode_bshd(&prm.tmap_v, a.v)) != CP_OK) return st;
+  if ((st = encode_in(&prm.tmap_q, a.q)) != CP_OK) return st;
+  if ((st = encode_in(&prm.tmap_k, a.k)) != CP_OK) return st;
+  if ((st = encode_in(&prm.tmap_v, a.v)) != CP_OK) return st;
   if ((st = encode_out(&prm.tmap_out, a.out)) != CP_OK) return st;
   prm.out = a.out.data;
   prm.out_bf16 = a.out.dtype == CP_BF16;
-  prm.o_sb = a.out.stride[0];
-  prm.o_ss = a.out.stride[1];
-  prm.o_sh = a.out.stride[2];
   prm.lse = static_cast<float*>(a.lse.data);
   prm.l_sb = a.lse.stride[0];
   prm.l_sh = a.lse.stride[1];
   prm.l_ss = a.lse.stride[2];
   prm.err = a.dev_err;
-  prm.B = (int)a.q.shape[0];
-  prm.S_q = (int)a.q.shape[1];
-  prm.H = (int)a.q.shape[2];
-  prm.S_kv = (int)a.k.shape[1];
+  if (a.q.ndim == 5) {   // [G, B, S/G, H, D] shards, read in place
+    prm.B = (int)a.q.shape[1];
+    prm.seg_q = (int)a.q.shape[2];
+    prm.S_q = (int)(a.q.shape[0] * a.q.shape[2]);
+    prm.H = (int)a.q.shape[3];
+    prm.seg_kv = (int)a.k.shape[2];
+    prm.S_kv = (int)(a.k.shape[0] * a.k.shape[2]);
+  } else {
+    prm.B = (int)a.q.shape[0];
+    prm.S_q = prm.seg_q = (int)a.q.shape[1];
+    prm.H = (int)a.q.shape[2];
+    prm.S_kv = prm.seg_kv = (int)a.k.shape[1];
+  }
+  if (prm.seg_q <= 0) prm.seg_q = 1;
+  if (prm.seg_kv <= 0) prm.seg_kv = 1;
   prm.n_q_blocks = (prm.S_q + 2 * kBlockM - 1) / (2 * kBlockM);
   prm.n_chunks = a.n_chunks;
   int n_tiles = 0;
@@ -562,7 +605,7 @@ int launch_attn_ring_tc(const RingArgs& a, cudaStream_t stream) {
   const long long grid = (long long)prm.n_q_blocks * prm.H * prm.B;
   if (grid <= 0 || n_tiles <= 0) return CP_OK;
   if (grid > 0x7fffffffLL) return CP_ERR_SHAPE;
-  const int D = (int)a.q.shape[3];
+  const int D = (int)a.q.shape[a.q.ndim - 1];
   if (D == 128) return launch_tc<128, kStagesD128>(prm, (int)grid, stream);
   if (D == 64) return launch_tc<64, kStagesD64>(prm, (int)grid, stream);
   return CP_ERR_SHAPE;

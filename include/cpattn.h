@@ -152,8 +152,13 @@ int cp_ulysses_permute(const cp_tensor* x, cp_tensor* y, int degree, int dir,
  *   q/k/v_shards, out_shards: [R*U, B, S/(R*U), H, D]
  *   lse: [B, H, S] f32 in token order (may be NULL)
  * Steps: Ulysses permute inside every group r; ring attention with R
- * chunks per head group u; inverse permute.  Intermediates live in the
- * caller's workspace (cp_usp_workspace_bytes); R = 1 is plain Ulysses.
+ * chunks per head group u; inverse permute.  R = 1 is plain Ulysses.
+ * For bf16 inputs with D in {64, 128}, 16-byte-aligned strides and a shard
+ * length S/(R*U) that is a multiple of 128, the permutations are folded into
+ * the attention kernel's tensor maps: one launch reads q/k/v and writes out
+ * in the shard layout, and the workspace is not used (may be NULL).
+ * Otherwise the intermediates live in the caller's workspace
+ * (cp_usp_workspace_bytes).
  */
 int cp_usp_attention(const cp_tensor* q_shards, const cp_tensor* k_shards,
                      const cp_tensor* v_shards, int ring_degree,
@@ -161,8 +166,10 @@ int cp_usp_attention(const cp_tensor* q_shards, const cp_tensor* k_shards,
                      size_t workspace_bytes, cp_tensor* out_shards,
                      cp_tensor* lse, void* stream);
 
-/* Workspace bytes cp_usp_attention needs for these sizes (0 on bad input).
- * in_dtype is the q/k/v dtype, out_dtype the out_shards dtype. */
+/* Workspace bytes cp_usp_attention needs for contiguous tensors of these
+ * sizes: 0 when the permutations fold into the attention kernel (see above)
+ * or on bad input.  in_dtype is the q/k/v dtype, out_dtype the out_shards
+ * dtype. */
 size_t cp_usp_workspace_bytes(int64_t B, int64_t S, int64_t H, int64_t D,
                               int in_dtype, int out_dtype, int ring_degree,
                               int ulysses_degree);

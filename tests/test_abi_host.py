@@ -132,12 +132,17 @@ def test_merge_errors():
 
 def test_usp_workspace_and_errors():
     L = bd.lib()
+    # shards of 2048 tokens (a multiple of 128): permutations fold into the
+    # attention kernel, no workspace
+    assert L.cp_usp_workspace_bytes(2, 8192, 24, 128, bd.CP_BF16, bd.CP_F32, 2, 2) == 0
+    # shards of 2050 tokens, or fp32 inputs: head-sharded q, k, v and out
+    n = 2 * 8200 * 24 * 128
+    assert L.cp_usp_workspace_bytes(2, 8200, 24, 128, bd.CP_BF16, bd.CP_F32, 2, 2) == 3 * n * 2 + n * 4
     n = 2 * 8192 * 24 * 128
-    need = L.cp_usp_workspace_bytes(2, 8192, 24, 128, bd.CP_BF16, bd.CP_F32, 2, 2)
-    assert need == 3 * n * 2 + n * 4
+    assert L.cp_usp_workspace_bytes(2, 8192, 24, 128, bd.CP_F32, bd.CP_F32, 2, 2) == 3 * n * 4 + n * 4
     assert L.cp_usp_workspace_bytes(2, 8192, 24, 128, 7, bd.CP_F32, 2, 2) == 0
     r = ctypes.byref
-    s = lambda off, dt=bd.CP_BF16: _t([4, 2, 2048, 24, 128], dt, FAKE + off)
+    s = lambda off, dt=bd.CP_BF16: _t([4, 2, 2050, 24, 128], dt, FAKE + off)
     q, k, v, o = s(0), s(1 << 30), s(2 << 30), s(3 << 30, bd.CP_F32)
     assert L.cp_usp_attention(r(q), r(k), r(v), 2, 2, 0.0, None, 0, r(o), None, None) == -9
     assert L.cp_usp_attention(r(q), r(k), r(v), 2, 2, 0.0, ctypes.c_void_p(FAKE), 16, r(o),
@@ -156,9 +161,9 @@ def test_static_scratch_entry_rejects_oversize_before_any_launch():
     fixed array, without touching the (fake) pointers or the GPU."""
     L = bd.lib()
     r = ctypes.byref
-    s = lambda off, dt=bd.CP_BF16: _t([4, 1, 2048, 24, 128], dt, FAKE + off)
+    s = lambda off, dt=bd.CP_BF16: _t([4, 1, 2050, 24, 128], dt, FAKE + off)
     q, k, v, o = s(0), s(1 << 30), s(2 << 30), s(3 << 30, bd.CP_F32)
-    need = L.cp_usp_workspace_bytes(1, 8192, 24, 128, bd.CP_BF16, bd.CP_F32, 2, 2)
+    need = L.cp_usp_workspace_bytes(1, 8200, 24, 128, bd.CP_BF16, bd.CP_F32, 2, 2)
     assert need > bd.USP_STATIC_SCRATCH_BYTES
     assert L.cp_usp_attention_static(r(q), r(k), r(v), 2, 2, 0.0, r(o), None, None) == -9
     assert L.cp_usp_attention_static(None, r(k), r(v), 2, 2, 0.0, r(o), None, None) == -1

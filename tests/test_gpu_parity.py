@@ -263,16 +263,22 @@ def test_workload_ulysses_and_unified_sampled(cuda_ok, R, U):
     _check(o_full, lse.cpu(), ro, rl, torch.bfloat16, rows=rows)
 
 
-def test_unified_small_matches_oracle_usp(cuda_ok):
-    """The emulated grid against the oracle's own rank-by-rank emulation."""
-    B, S, H, D, R, U = 2, 512, 8, 128, 2, 2
-    q, k, v = wl.make_qkv(B, H, S, D, torch.bfloat16, 19)
+@pytest.mark.parametrize("S,D,dtype", [(512, 128, torch.bfloat16),    # shards of 128: fused
+                                       (600, 64, torch.bfloat16),     # shards of 150: permute path
+                                       (1000, 128, torch.bfloat16),   # shards of 250: permute path
+                                       (264, 64, torch.float32)])     # fp32: permute path
+def test_unified_small_matches_oracle_usp(cuda_ok, S, D, dtype):
+    """The emulated grid against the oracle's own rank-by-rank emulation,
+    through both the fused (tensor-map) path and the permute path."""
+    B, H, R, U = 2, 8, 2, 2
+    q, k, v = wl.make_qkv(B, H, S, D, dtype, 19)
     sh = lambda t: wl.sequence_shards(t, R * U)
     out, lse = cp.usp_attention(*_dev(sh(q), sh(k), sh(v)), R, U)
     torch.cuda.synchronize()
     ro, rl = oracle.usp_attention(_np(sh(q)), _np(sh(k)), _np(sh(v)), R, U)
-    assert np.abs(_np(out) - ro).max() <= 2e-2
-    assert np.abs(_np(lse) - rl).max() <= 1e-3
+    tol_o, tol_l = TOL[dtype]
+    assert np.abs(_np(out) - ro).max() <= tol_o
+    assert np.abs(_np(lse) - rl).max() <= tol_l
 
 
 # ---------------------------------------------------------------- failure surfacing
