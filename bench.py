@@ -308,6 +308,21 @@ def run_cuda(args):
         components[name] = {"shape": list(x.shape), "bytes": pbytes, "ms": float(np.mean(t_p)),
                             "GB/s": gbs, "frac_of_hbm": gbs / hbm_peak}
     del x, y, x2, oi, li, acc, lacc
+    # unified R=2 x U=2 grid (B=2, S=8192, H=24, D=128) from sequence shards
+    uq, uk, uv = wl.make_workload_inputs(u)
+    ush = [wl.sequence_shards(t, 4).to(dev) for t in (uq, uk, uv)]
+    del uq, uk, uv
+    uout = torch.empty(ush[0].shape, dtype=torch.float32, device=dev)
+    uws = torch.empty(max(1, cp.usp_workspace_bytes(u.B, u.S, u.H, u.D, torch.bfloat16,
+                                                    torch.float32, 2, 2)),
+                      dtype=torch.uint8, device=dev)
+    t_u = _time_loop(lambda: cp.usp_attention(*ush, 2, 2, out=uout, workspace=uws,
+                                              want_lse=False), n_merge, 3, flush, stream)
+    tf = u.flops / (np.mean(t_u) * 1e-3) / 1e12
+    components["usp_attention_R2_U2"] = {"shape": list(ush[0].shape), "flops": u.flops,
+                                         "ms": float(np.mean(t_u)), "TFLOP/s": tf,
+                                         "frac_of_bf16_peak": tf / tc_peak}
+    del ush, uout, uws
     if args.extra:
         components.update(_extra_workloads(cp, wl, dev, stream, flush, tc_peak))
 
