@@ -16,7 +16,9 @@ Everything here is the plain definition, written out in float64 NumPy:
 * ``lse_merge``          the fp32-style merge of two (out, lse) partials;
 * ``ring_attention``     the literal ring walk: partial per chunk + merge;
 * ``ulysses_permute``    the sequence-shard <-> head-shard all-to-all index map;
-* ``usp_attention``      the unified (Ulysses x Ring) composition.
+* ``usp_attention``      the unified (Ulysses x Ring) composition;
+* ``ulysses_anything_*``  the all-to-all and attention with uneven sequence
+                         and head splits (Ulysses Anything).
 
 Pins: every function is checked in ``tests/test_oracle.py`` against facts
 that do not come from the oracle itself (closed forms, brute force loops on
@@ -25,10 +27,12 @@ worked examples in ``tests/golden/``).  No function is left parity-unpinned.
 """
 from .attention import (attention, attention_partial, attention_bruteforce,
                         lse_merge, ring_attention, ring_chunk_offsets)
-from .ulysses import ulysses_permute, ulysses_permute_bruteforce, usp_attention
+from .ulysses import (ulysses_permute, ulysses_permute_bruteforce, usp_attention,
+                      uneven_offsets, ulysses_anything_permute, ulysses_anything_attention)
 
 __all__ = [
     "attention", "attention_partial", "attention_bruteforce", "lse_merge",
     "ring_attention", "ring_chunk_offsets", "ulysses_permute",
-    "ulysses_permute_bruteforce", "usp_attention",
+    "ulysses_permute_bruteforce", "usp_attention", "uneven_offsets",
+    "ulysses_anything_permute", "ulysses_anything_attention",
 ]

@@ -15,6 +15,9 @@ Sources, by page and section:
   one Ring group.
 * diffusers parallelism API page, §ContextParallelConfig ``mesh``: the mesh
   dimensions are named ("ring", "ulysses", ...) in that order.
+* same guide, §Ulysses Anything Attention (and ContextParallelConfig
+  ``ulysses_anything``): sequence lengths and head counts that the degree
+  does not divide are accepted; ring_degree must be 1.
 
 Readings (the pages give no index map): shards are held rank-major as one
 [U, B, S/U, H, D] tensor; head group q is the contiguous heads
@@ -137,4 +140,77 @@ def usp_attention(q_shards, k_shards, v_shards, ring_degree: int, ulysses_degree
             lse[:, u * Hg:(u + 1) * Hg, r * SR:(r + 1) * SR] = acc_l
     # step 3: inverse all-to-all inside every group r
     out = np.concatenate([ulysses_permute(o[r], U, HEAD_TO_SEQ) for r in range(R)], axis=0)
+    return out, lse
+
+
+# ---------------------------------------------------------------- Ulysses Anything
+def uneven_offsets(n: int, degree: int):
+    """Offsets [0, ..., n] of `degree` ranks holding ceil(n/degree) items
+    each, the last ranks holding what is left (possibly nothing).  The guide's
+    Ulysses Anything section accepts sequence lengths and head counts that
+    the degree does not divide; this even-as-possible split is the plain
+    reading (the same rule as the Ring Anything chunks)."""
+    c = -(-n // degree) if n > 0 else 0
+    offs = [0]
+    for _ in range(degree):
+        offs.append(min(n, offs[-1] + c))
+    return offs
+
+
+def ulysses_anything_permute(x, B: int, H: int, D: int, seq_offsets, head_offsets,
+                             direction: int) -> np.ndarray:
+    """Ulysses Anything all-to-all on flat per-rank buffers.
+
+    Sequence side: the concatenation of U rank buffers, rank p holding
+    [B, s_p, H, D] with s_p = seq_offsets[p+1] - seq_offsets[p].
+    Head side: the concatenation of U rank buffers, rank q holding
+    [B, S, h_q, D] (all S tokens in order) with h_q from head_offsets.
+    direction 0: y[q][b, off_p + s, h', d] = x[p][b, s, hoff_q + h', d];
+    direction 1 is the exact inverse.  Pure data movement.
+    """
+    U = len(seq_offsets) - 1
+    S = seq_offsets[-1]
+    x = np.asarray(x).reshape(-1)
+    y = np.empty_like(x)
+    for q in range(U):
+        h0, h1 = head_offsets[q], head_offsets[q + 1]
+        hq = h1 - h0
+        ybase = B * S * h0 * D
+        for p in range(U):
+            s0, s1 = seq_offsets[p], seq_offsets[p + 1]
+            sp = s1 - s0
+            xbase = B * s0 * H * D
+            seq_blk = (slice(xbase, xbase + B * sp * H * D), (B, sp, H, D))
+            head_blk = (slice(ybase, ybase + B * S * hq * D), (B, S, hq, D))
+            if direction == SEQ_TO_HEAD:
+                src = x[seq_blk[0]].reshape(seq_blk[1])
+                y[head_blk[0]].reshape(head_blk[1])[:, s0:s1] = src[:, :, h0:h1]
+            else:
+                src = x[head_blk[0]].reshape(head_blk[1])
+                y[seq_blk[0]].reshape(seq_blk[1])[:, :, h0:h1] = src[:, s0:s1]
+    return y
+
+
+def ulysses_anything_attention(q_flat, k_flat, v_flat, B: int, H: int, D: int, seq_offsets,
+                               head_offsets, scale: Optional[float] = None):
+    """Ulysses Anything (ring_degree 1): all-to-all to uneven head groups,
+    attention of every head group over the whole sequence, inverse
+    all-to-all.  Returns the flat sequence-sharded output and the lse of
+    every query as [B, H, S] (token order), float64."""
+    S = seq_offsets[-1]
+    U = len(seq_offsets) - 1
+    yq, yk, yv = (ulysses_anything_permute(np.asarray(t, dtype=np.float64), B, H, D,
+                                           seq_offsets, head_offsets, SEQ_TO_HEAD)
+                  for t in (q_flat, k_flat, v_flat))
+    yo = np.empty_like(yq)
+    lse = np.full((B, H, S), -np.inf)
+    for q in range(U):
+        h0, h1 = head_offsets[q], head_offsets[q + 1]
+        hq = h1 - h0
+        sl = slice(B * S * h0 * D, B * S * h1 * D)
+        o, l = attention_partial(yq[sl].reshape(B, S, hq, D), yk[sl].reshape(B, S, hq, D),
+                                 yv[sl].reshape(B, S, hq, D), scale)
+        yo[sl] = o.reshape(-1)
+        lse[:, h0:h1] = l
+    out = ulysses_anything_permute(yo, B, H, D, seq_offsets, head_offsets, HEAD_TO_SEQ)
     return out, lse

@@ -308,3 +308,57 @@ def test_planted_permute_mistake_is_caught():
     assert not np.array_equal(shard_order_swapped(x, 2, 0), y)
     x3 = np.arange(2 * 1 * 2 * 4 * 1).reshape(2, 1, 2, 4, 1)
     assert not np.array_equal(head_major_wrong(x3, 2, 0), oracle.ulysses_permute_bruteforce(x3, 2, 0))
+
+
+# ---------------------------------------------------------------- Ulysses Anything
+def _flat_shards(full, offs):
+    """Rank buffers of a [B, S, H, D] array split at `offs`, concatenated."""
+    return np.concatenate([full[:, offs[p]:offs[p + 1]].reshape(-1) for p in range(len(offs) - 1)])
+
+
+def test_uneven_offsets_rule():
+    assert oracle.uneven_offsets(4481, 4) == [0, 1121, 2242, 3363, 4481]
+    assert oracle.uneven_offsets(24, 5) == [0, 5, 10, 15, 20, 24]
+    assert oracle.uneven_offsets(3, 4) == [0, 1, 2, 3, 3]
+
+
+def test_ulysses_anything_reduces_to_even_map():
+    """With even splits the flat rank buffers are exactly the rank-major
+    tensors of the even all-to-all, so both maps must agree bit for bit."""
+    U, B, S, H, D = 4, 2, 16, 8, 3
+    x = np.arange(B * S * H * D).reshape(B, S, H, D)
+    so, ho = oracle.uneven_offsets(S, U), oracle.uneven_offsets(H, U)
+    flat = _flat_shards(x, so)
+    even = x.reshape(B, U, S // U, H, D).transpose(1, 0, 2, 3, 4)
+    y = oracle.ulysses_anything_permute(flat, B, H, D, so, ho, 0)
+    assert np.array_equal(y, oracle.ulysses_permute(even, U, 0).reshape(-1))
+
+
+@pytest.mark.parametrize("U,B,S,H,D", [(4, 1, 13, 6, 2), (5, 2, 11, 24, 1), (3, 1, 7, 4, 3)])
+def test_ulysses_anything_bruteforce_and_inverse(U, B, S, H, D):
+    so, ho = oracle.uneven_offsets(S, U), oracle.uneven_offsets(H, U)
+    full = np.arange(B * S * H * D).reshape(B, S, H, D)
+    x = _flat_shards(full, so)
+    y = oracle.ulysses_anything_permute(x, B, H, D, so, ho, 0)
+    # element by element: rank q holds every token of its heads, in order
+    pos = 0
+    for q in range(U):
+        for b in range(B):
+            for t in range(S):
+                for h in range(ho[q], ho[q + 1]):
+                    for d in range(D):
+                        assert y[pos] == full[b, t, h, d]
+                        pos += 1
+    assert np.array_equal(oracle.ulysses_anything_permute(y, B, H, D, so, ho, 1), x)
+
+
+@pytest.mark.parametrize("U,S,H", [(4, 37, 8), (5, 23, 24), (3, 19, 7)])
+def test_ulysses_anything_attention_equals_oneshot(U, S, H):
+    B, D = 2, 8
+    q, k, v = _qkv(B, H, S, S, D, 200 + U)
+    so, ho = oracle.uneven_offsets(S, U), oracle.uneven_offsets(H, U)
+    out, lse = oracle.ulysses_anything_attention(_flat_shards(q, so), _flat_shards(k, so),
+                                                 _flat_shards(v, so), B, H, D, so, ho)
+    o, l = oracle.attention(q, k, v)
+    np.testing.assert_allclose(out, _flat_shards(o, so), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse, l, rtol=0, atol=1e-13)
