@@ -323,6 +323,27 @@ def run_cuda(args):
                                          "ms": float(np.mean(t_u)), "TFLOP/s": tf,
                                          "frac_of_bf16_peak": tf / tc_peak}
     del ush, uout, uws
+    # Ulysses Anything on FLUX at 1008x1008: 3969 + 512 = 4481 tokens, U = 4
+    # (1121, 1121, 1121, 1118 tokens per rank; 6 heads each)
+    A_S, A_U = 4481, 4
+    aq, ak, av = wl.make_qkv(1, 24, A_S, 128, torch.bfloat16, 1101, "kscale")
+    so = cp.ring_chunk_offsets(A_S, A_U)
+    ho = cp.ring_chunk_offsets(24, A_U)
+    flat = lambda t: torch.cat([t[:, so[p]:so[p + 1]].reshape(-1) for p in range(A_U)]).to(dev)
+    aq, ak, av = flat(aq), flat(ak), flat(av)
+    aout = torch.empty(aq.shape, dtype=torch.float32, device=dev)
+    aws = torch.empty(cp.binding.lib().cp_ulysses_anything_workspace_bytes(
+        1, A_S, 24, 128, cp.binding.CP_BF16, cp.binding.CP_F32), dtype=torch.uint8, device=dev)
+    t_a = _time_loop(lambda: cp.ulysses_anything_attention(aq, ak, av, 1, 24, 128, so, ho,
+                                                           out=aout, workspace=aws,
+                                                           want_lse=False),
+                     n_merge, 3, flush, stream)
+    aflops = 4.0 * 24 * A_S * A_S * 128
+    tf = aflops / (np.mean(t_a) * 1e-3) / 1e12
+    components["ulysses_anything_1008px_U4"] = {"S": A_S, "flops": aflops,
+                                                "ms": float(np.mean(t_a)), "TFLOP/s": tf,
+                                                "frac_of_bf16_peak": tf / tc_peak}
+    del aq, ak, av, aout, aws
     if args.extra:
         components.update(_extra_workloads(cp, wl, dev, stream, flush, tc_peak))
 

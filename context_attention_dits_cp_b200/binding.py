@@ -30,7 +30,8 @@ STATUS = {
 }
 EXPORTS = ("cp_attn_partial", "cp_lse_merge", "cp_ring_attention", "cp_ulysses_permute",
            "cp_usp_attention", "cp_usp_attention_static", "cp_usp_workspace_bytes",
-           "cp_ring_chunk_offsets",
+           "cp_ulysses_anything_permute", "cp_ulysses_anything_attention",
+           "cp_ulysses_anything_workspace_bytes", "cp_ring_chunk_offsets",
            "cp_status_string", "cp_last_device_error", "cp_selftest_wait_timeout")
 
 
@@ -69,12 +70,19 @@ def lib() -> ctypes.CDLL:
         L.cp_usp_workspace_bytes.argtypes = [i64, i64, i64, i64, i32, i32, i32, i32]
         L.cp_usp_workspace_bytes.restype = ctypes.c_size_t
         L.cp_ring_chunk_offsets.argtypes = [i64, i32, ctypes.POINTER(i64)]
+        OFF = ctypes.POINTER(i64)
+        L.cp_ulysses_anything_permute.argtypes = [P, P, i64, i64, i64, i32, OFF, OFF, i32, vp]
+        L.cp_ulysses_anything_attention.argtypes = [P, P, P, i64, i64, i64, i32, OFF, OFF, f32,
+                                                    vp, ctypes.c_size_t, P, P, vp]
+        L.cp_ulysses_anything_workspace_bytes.argtypes = [i64, i64, i64, i64, i32, i32]
+        L.cp_ulysses_anything_workspace_bytes.restype = ctypes.c_size_t
         L.cp_status_string.argtypes = [i32]
         L.cp_status_string.restype = ctypes.c_char_p
         L.cp_last_device_error.argtypes = [vp]
         L.cp_selftest_wait_timeout.argtypes = [i32, vp]
         for n in EXPORTS:
-            if n not in ("cp_usp_workspace_bytes", "cp_status_string"):
+            if n not in ("cp_usp_workspace_bytes", "cp_status_string",
+                         "cp_ulysses_anything_workspace_bytes"):
                 getattr(L, n).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -199,6 +207,44 @@ def usp_attention(q_shards, k_shards, v_shards, ring_degree: int, ulysses_degree
                                   ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
                                   _ref(do), _ref(dl), _stream(q_shards.device)),
            "cp_usp_attention")
+    return out, lse
+
+
+def _offsets(offs):
+    return (ctypes.c_int64 * len(offs))(*[int(x) for x in offs])
+
+
+def ulysses_anything_permute(x, B, H, D, seq_offsets, head_offsets, direction, y=None):
+    """Uneven Ulysses all-to-all on flat rank buffers (cp_ulysses_anything_permute)."""
+    y = torch.empty_like(x) if y is None else y
+    U = len(seq_offsets) - 1
+    _check(lib().cp_ulysses_anything_permute(_ref(desc(x)), _ref(desc(y)), int(B), int(H), int(D),
+                                             U, _offsets(seq_offsets), _offsets(head_offsets),
+                                             int(direction), _stream(x.device)),
+           "cp_ulysses_anything_permute")
+    return y
+
+
+def ulysses_anything_attention(q, k, v, B, H, D, seq_offsets, head_offsets, scale=None,
+                               out=None, lse=None, workspace=None, out_dtype=torch.float32,
+                               want_lse=True):
+    """Ulysses Anything attention on flat sequence-side buffers
+    (cp_ulysses_anything_attention)."""
+    S = int(seq_offsets[-1])
+    U = len(seq_offsets) - 1
+    out = torch.empty(q.shape, dtype=out_dtype, device=q.device) if out is None else out
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        code = lambda dt: CP_F32 if dt == torch.float32 else CP_BF16
+        need = int(lib().cp_ulysses_anything_workspace_bytes(B, S, H, D, code(q.dtype),
+                                                             code(out.dtype)))
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _check(lib().cp_ulysses_anything_attention(
+        _ref(desc(q)), _ref(desc(k)), _ref(desc(v)), int(B), int(H), int(D), U,
+        _offsets(seq_offsets), _offsets(head_offsets), _scale(scale),
+        ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _ref(desc(out)),
+        _ref(desc(lse)), _stream(q.device)), "cp_ulysses_anything_attention")
     return out, lse
 
 

@@ -409,6 +409,155 @@ int cp_usp_attention(const cp_tensor* qs, const cp_tensor* ks, const cp_tensor* 
   return CP_OK;
 }
 
+}  // extern "C"
+
+namespace cpattn {
+namespace {
+// n+1 host offsets starting at 0, non-decreasing, ending at `total`.
+int check_offsets(const int64_t* off, int n, int64_t total) {
+  if (!off) return CP_ERR_NULL;
+  if (off[0] != 0 || off[n] != total) return CP_ERR_OFFSETS;
+  for (int i = 0; i < n; ++i)
+    if (off[i + 1] < off[i]) return CP_ERR_OFFSETS;
+  return CP_OK;
+}
+
+// Flat contiguous 1-D buffer of `n` elements.
+int check_flat(const cp_tensor* t, int64_t n) {
+  int st;
+  if ((st = check_basic(t, 1))) return st;
+  if (t->shape[0] != n) return CP_ERR_SHAPE;
+  if (n > 1 && t->stride[0] != 1) return CP_ERR_ALIGN;
+  return CP_OK;
+}
+
+cp_tensor flat_view(void* data, int dtype, int64_t n) {
+  cp_tensor t;
+  memset(&t, 0, sizeof(t));
+  t.data = data;
+  t.dtype = dtype;
+  t.ndim = 1;
+  t.shape[0] = n;
+  t.stride[0] = 1;
+  return t;
+}
+}  // namespace
+}  // namespace cpattn
+
+extern "C" {
+
+int cp_ulysses_anything_permute(const cp_tensor* x, cp_tensor* y, int64_t B, int64_t H,
+                                int64_t D, int degree, const int64_t* seq_offsets,
+                                const int64_t* head_offsets, int dir, void* stream) {
+  int st;
+  if (degree < 1 || degree > CP_MAX_CHUNKS) return CP_ERR_DEGREE;
+  if (dir != 0 && dir != 1) return CP_ERR_SHAPE;
+  if (B < 0 || H < 0 || D < 1) return CP_ERR_SHAPE;
+  if (!seq_offsets || !head_offsets) return CP_ERR_NULL;
+  const int64_t S = seq_offsets[degree];
+  if (S < 0 || S > 0x7fffffffLL || H > 0x7fffffffLL) return CP_ERR_SHAPE;
+  if ((st = check_offsets(seq_offsets, degree, S)) || (st = check_offsets(head_offsets, degree, H)))
+    return st;
+  const int64_t n = B * S * H * D;
+  if ((st = check_flat(x, n)) || (st = check_flat(y, n))) return st;
+  if (x->dtype != y->dtype) return CP_ERR_DTYPE;
+  const TensorView vx = view_of(x), vy = view_of(y);
+  if (overlaps(vx, vy)) return CP_ERR_ALIAS;
+  if (n == 0) return CP_OK;
+  return launch_ulysses_anything_permute(vx, vy, B, H, D, degree, seq_offsets, head_offsets, dir,
+                                         as_stream(stream));
+}
+
+size_t cp_ulysses_anything_workspace_bytes(int64_t B, int64_t S, int64_t H, int64_t D,
+                                           int in_dtype, int out_dtype) {
+  if (B < 0 || S < 0 || H < 0 || D < 0) return 0;
+  if (B == 1) return 0;   // the rank buffers are read in place
+  if ((in_dtype != CP_F32 && in_dtype != CP_BF16) || (out_dtype != CP_F32 && out_dtype != CP_BF16))
+    return 0;
+  return usp_unfused_bytes(B, S, H, D, in_dtype, out_dtype);
+}
+
+int cp_ulysses_anything_attention(const cp_tensor* q, const cp_tensor* k, const cp_tensor* v,
+                                  int64_t B, int64_t H, int64_t D, int degree,
+                                  const int64_t* seq_offsets, const int64_t* head_offsets,
+                                  float scale, void* workspace, size_t workspace_bytes,
+                                  cp_tensor* out, cp_tensor* lse, void* stream) {
+  int st;
+  if (degree < 1 || degree > CP_MAX_CHUNKS) return CP_ERR_DEGREE;
+  if (B < 0 || H < 0 || (D != 64 && D != 128)) return CP_ERR_SHAPE;
+  if (!seq_offsets || !head_offsets) return CP_ERR_NULL;
+  const int64_t S = seq_offsets[degree];
+  if (S < 0 || S > 0x7fffffffLL || H > 0x7fffffffLL) return CP_ERR_SHAPE;
+  if ((st = check_offsets(seq_offsets, degree, S)) || (st = check_offsets(head_offsets, degree, H)))
+    return st;
+  const int64_t n = B * S * H * D;
+  if ((st = check_flat(q, n)) || (st = check_flat(k, n)) || (st = check_flat(v, n)) ||
+      (st = check_flat(out, n)))
+    return st;
+  if (q->dtype != k->dtype || q->dtype != v->dtype) return CP_ERR_DTYPE;
+  if (lse) {
+    if ((st = check_basic(lse, 3))) return st;
+    if (lse->dtype != CP_F32) return CP_ERR_DTYPE;
+    if (lse->shape[0] != B || lse->shape[1] != H || lse->shape[2] != S) return CP_ERR_SHAPE;
+  }
+  const TensorView vo = view_of(out);
+  if (overlaps(vo, view_of(q)) || overlaps(vo, view_of(k)) || overlaps(vo, view_of(v)))
+    return CP_ERR_ALIAS;
+  if (n == 0) return CP_OK;
+
+  // On one GPU every head group sits on the same device, and attention of
+  // each head group over the whole sequence is attention over all heads: so
+  // the all-to-all is carried out only as far as the attention kernel needs.
+  // Rank buffers [B, s_p, H, D] concatenated in rank order are, for B = 1,
+  // already one contiguous [1, S, H, D] tensor, read in place; for B > 1 an
+  // uneven all-to-all whose single head group holds all H heads gathers the
+  // sequence into [B, S, H, D] (and its inverse scatters the output back).
+  const int64_t one[2] = {0, S};
+  auto bshd = [&](void* data, int dtype) {
+    cp_tensor t;
+    memset(&t, 0, sizeof(t));
+    t.data = data;
+    t.dtype = dtype;
+    t.ndim = 4;
+    const int64_t sh[4] = {B, S, H, D};
+    const int64_t sd[4] = {S * H * D, H * D, D, 1};
+    for (int j = 0; j < 4; ++j) {
+      t.shape[j] = sh[j];
+      t.stride[j] = sd[j];
+    }
+    return t;
+  };
+  if (B == 1) {
+    cp_tensor t4[4] = {bshd(q->data, q->dtype), bshd(k->data, k->dtype), bshd(v->data, v->dtype),
+                       bshd(out->data, out->dtype)};
+    return ring_impl(&t4[0], &t4[1], &t4[2], one, 1, scale, &t4[3], lse, stream);
+  }
+  if (!workspace) return CP_ERR_WORKSPACE;
+  if (workspace_bytes < usp_unfused_bytes(B, S, H, D, q->dtype, out->dtype))
+    return CP_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return CP_ERR_ALIGN;
+  auto rnd = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  const int esi = dtype_size(q->dtype);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* Y[3] = {ws, ws + rnd(n * esi), ws + 2 * rnd(n * esi)};
+  uint8_t* Yo = ws + 3 * rnd(n * esi);
+  int64_t all_heads[CP_MAX_CHUNKS + 1];
+  all_heads[0] = 0;
+  for (int g = 1; g <= degree; ++g) all_heads[g] = H;
+  const cp_tensor* ins[3] = {q, k, v};
+  for (int i = 0; i < 3; ++i) {
+    cp_tensor y = flat_view(Y[i], q->dtype, n);
+    if ((st = cp_ulysses_anything_permute(ins[i], &y, B, H, D, degree, seq_offsets, all_heads, 0,
+                                          stream)))
+      return st;
+  }
+  cp_tensor t4[4] = {bshd(Y[0], q->dtype), bshd(Y[1], q->dtype), bshd(Y[2], q->dtype),
+                     bshd(Yo, out->dtype)};
+  if ((st = ring_impl(&t4[0], &t4[1], &t4[2], one, 1, scale, &t4[3], lse, stream))) return st;
+  cp_tensor yo = flat_view(Yo, out->dtype, n);
+  return cp_ulysses_anything_permute(&yo, out, B, H, D, degree, seq_offsets, all_heads, 1, stream);
+}
+
 int cp_ring_chunk_offsets(int64_t S, int R, int64_t* offsets) {
   if (!offsets) return CP_ERR_NULL;
   if (S < 0 || R < 1) return CP_ERR_SHAPE;

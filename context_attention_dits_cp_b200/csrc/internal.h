@@ -50,6 +50,9 @@ int launch_lse_merge(const TensorView& out_acc, const TensorView& lse_acc,
                      const TensorView& out_i, const TensorView& lse_i, cudaStream_t stream);
 int launch_ulysses_permute(const TensorView& x, const TensorView& y, int degree, int dir,
                            cudaStream_t stream);
+int launch_ulysses_anything_permute(const TensorView& x, const TensorView& y, int64_t B,
+                                    int64_t H, int64_t D, int U, const int64_t* seq_off,
+                                    const int64_t* head_off, int dir, cudaStream_t stream);
 int launch_wait_timeout_selftest(int spin_limit, int* dev_err, cudaStream_t stream);
 
 }  // namespace cpattn

@@ -203,6 +203,51 @@ int cp_usp_attention_static(const cp_tensor* q_shards,
                             void* stream);
 
 /*
+ * cp_ulysses_anything_permute -- the Ulysses all-to-all when the degree U
+ * divides neither the sequence length nor the head count (§Ulysses Anything
+ * Attention; ContextParallelConfig.ulysses_anything).  Rank p holds tokens
+ * [seq_offsets[p], seq_offsets[p+1]), rank q heads [head_offsets[q],
+ * head_offsets[q+1]) (HOST arrays of U+1 int64: 0, non-decreasing, ending
+ * at S and H; cp_ring_chunk_offsets gives the ceil split).  Every rank's
+ * buffer is contiguous, so both sides are flat 1-D buffers of B*S*H*D
+ * elements, the rank buffers concatenated in rank order:
+ *   sequence side: rank p holds [B, s_p, H, D]
+ *   head side:     rank q holds [B, S, h_q, D] (every token, in order)
+ *   dir 0: y[q][b, off_p + s, h', d] = x[p][b, s, hoff_q + h', d]
+ *   dir 1: the exact inverse.
+ * Bit-exact copy; x and y same dtype, contiguous, not overlapping.
+ * 1 <= U <= CP_MAX_CHUNKS; empty ranks are allowed.
+ */
+int cp_ulysses_anything_permute(const cp_tensor* x, cp_tensor* y, int64_t B,
+                                int64_t H, int64_t D, int degree,
+                                const int64_t* seq_offsets,
+                                const int64_t* head_offsets, int dir,
+                                void* stream);
+
+/*
+ * cp_ulysses_anything_attention -- Ulysses Anything (ring_degree 1): the
+ * uneven all-to-all above, attention of every head group over the whole
+ * sequence, and the inverse all-to-all.  q/k/v/out are flat sequence-side
+ * buffers as above (out f32 or bf16); lse is [B, H, S] f32 in token order
+ * (may be NULL).  On one GPU all head groups share the device, so the data
+ * is moved only as far as one attention launch over all heads needs: for
+ * B = 1 the rank buffers already form [1, S, H, D] and are read in place
+ * (no workspace); for B > 1 the sequence is gathered into the caller's
+ * workspace of cp_ulysses_anything_workspace_bytes bytes (256-byte
+ * aligned) and the output scattered back.
+ */
+int cp_ulysses_anything_attention(const cp_tensor* q, const cp_tensor* k,
+                                  const cp_tensor* v, int64_t B, int64_t H,
+                                  int64_t D, int degree,
+                                  const int64_t* seq_offsets,
+                                  const int64_t* head_offsets, float scale,
+                                  void* workspace, size_t workspace_bytes,
+                                  cp_tensor* out, cp_tensor* lse, void* stream);
+size_t cp_ulysses_anything_workspace_bytes(int64_t B, int64_t S, int64_t H,
+                                           int64_t D, int in_dtype,
+                                           int out_dtype);
+
+/*
  * cp_ring_chunk_offsets -- the Ring Anything split of S tokens over R ranks:
  * ceil(S/R) tokens per rank, the last ranks holding the rest (possibly
  * nothing).  Writes R+1 offsets to the HOST array `offsets`.

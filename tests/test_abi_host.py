@@ -167,3 +167,33 @@ def test_static_scratch_entry_rejects_oversize_before_any_launch():
     assert need > bd.USP_STATIC_SCRATCH_BYTES
     assert L.cp_usp_attention_static(r(q), r(k), r(v), 2, 2, 0.0, r(o), None, None) == -9
     assert L.cp_usp_attention_static(None, r(k), r(v), 2, 2, 0.0, r(o), None, None) == -1
+
+
+def test_ulysses_anything_argument_errors():
+    L = bd.lib()
+    r = ctypes.byref
+    B, H, D = 1, 24, 128
+    so, ho = [0, 1121, 2242, 3363, 4481], [0, 6, 12, 18, 24]
+    n = B * 4481 * H * D
+    x, y = _t([n], data=FAKE), _t([n], data=FAKE + (1 << 30))
+    off = lambda a: (ctypes.c_int64 * len(a))(*a)
+    call = lambda xs, ys, s_, h_, dr=0, dg=4: L.cp_ulysses_anything_permute(
+        r(xs), r(ys), B, H, D, dg, off(s_), off(h_), dr, None)
+    assert call(x, y, [1, 1121, 2242, 3363, 4481], ho) == -5      # must start at 0
+    assert call(x, y, [0, 1121, 1000, 3363, 4481], ho) == -5      # monotone
+    assert call(x, y, so, [0, 6, 12, 18, 23]) == -5               # heads must end at H
+    assert call(x, _t([n - 1], data=FAKE + (1 << 30)), so, ho) == -3
+    assert call(x, _t([n], bd.CP_F32, FAKE + (1 << 30)), so, ho) == -2
+    assert call(x, _t([n], data=FAKE + 64), so, ho) == -10        # overlap
+    assert call(x, y, so, ho, dr=2) == -3
+    assert call(x, y, so, ho, dg=0) == -6
+    assert L.cp_ulysses_anything_workspace_bytes(1, 4481, 24, 128, bd.CP_BF16, bd.CP_F32) == 0
+    n2 = 2 * n
+    assert L.cp_ulysses_anything_workspace_bytes(2, 4481, 24, 128, bd.CP_BF16, bd.CP_F32) == \
+        3 * ((n2 * 2 + 255) // 256 * 256) + (n2 * 4 + 255) // 256 * 256
+    q, k, v = _t([n2], data=FAKE), _t([n2], data=FAKE + (1 << 30)), _t([n2], data=FAKE + (2 << 30))
+    o = _t([n2], bd.CP_F32, FAKE + (3 << 30))
+    att = lambda ws, wsb: L.cp_ulysses_anything_attention(
+        r(q), r(k), r(v), 2, H, D, 4, off(so), off(ho), 0.0, ws, wsb, r(o), None, None)
+    assert att(None, 0) == -9
+    assert att(ctypes.c_void_p(FAKE), 1024) == -9

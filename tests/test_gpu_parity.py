@@ -281,6 +281,66 @@ def test_unified_small_matches_oracle_usp(cuda_ok, S, D, dtype):
     assert np.abs(_np(lse) - rl).max() <= tol_l
 
 
+# ---------------------------------------------------------------- Ulysses Anything
+def _flat(full, offs):
+    return torch.cat([full[:, offs[p]:offs[p + 1]].reshape(-1) for p in range(len(offs) - 1)])
+
+
+def _unflat(flat, offs, B, H, D):
+    parts, pos = [], 0
+    for p in range(len(offs) - 1):
+        n = B * (offs[p + 1] - offs[p]) * H * D
+        parts.append(flat[pos:pos + n].reshape(B, offs[p + 1] - offs[p], H, D))
+        pos += n
+    return torch.cat(parts, dim=1)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("B,S,H,D,U", [(1, 4481, 24, 128, 4),   # FLUX at 1008x1008
+                                       (2, 37, 24, 64, 5),      # uneven heads 5,5,5,5,4
+                                       (1, 10, 3, 64, 4)])      # an empty head group
+def test_ulysses_anything_permute_bit_exact(cuda_ok, dtype, B, S, H, D, U):
+    so, ho = oracle.uneven_offsets(S, U), oracle.uneven_offsets(H, U)
+    x = _flat(torch.randn(B, S, H, D).to(dtype), so)
+    y = cp.ulysses_anything_permute(x.cuda(), B, H, D, so, ho, cp.SEQ_TO_HEAD)
+    torch.cuda.synchronize()
+    iv = torch.int16 if dtype == torch.bfloat16 else torch.int32
+    bits = lambda t: t.cpu().view(iv).numpy()
+    assert np.array_equal(bits(y), oracle.ulysses_anything_permute(bits(x), B, H, D, so, ho, 0))
+    x2 = cp.ulysses_anything_permute(y, B, H, D, so, ho, cp.HEAD_TO_SEQ)
+    assert np.array_equal(bits(x2), bits(x))
+
+
+def test_ulysses_anything_attention_1008px_sampled(cuda_ok):
+    """FLUX at 1008x1008: 3969 image + 512 text tokens on 4 ranks, where the
+    guide's plain Ulysses fails and Ulysses Anything runs."""
+    B, S, H, D, U = 1, 4481, 24, 128, 4
+    q, k, v = wl.make_qkv(B, H, S, D, torch.bfloat16, 41, "kscale")
+    so, ho = oracle.uneven_offsets(S, U), oracle.uneven_offsets(H, U)
+    out, lse = cp.ulysses_anything_attention(*(_flat(t, so).cuda() for t in (q, k, v)),
+                                             B, H, D, so, ho)
+    torch.cuda.synchronize()
+    o_full = _unflat(out.cpu(), so, B, H, D)
+    rows = _rows(S, 48, 6)
+    ro, rl = oracle.attention(_np(q), _np(k), _np(v), rows=rows)
+    _check(o_full, lse.cpu(), ro, rl, torch.bfloat16, rows=rows)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("S,H,U", [(300, 6, 4), (129, 24, 5)])
+def test_ulysses_anything_attention_matches_oracle(cuda_ok, dtype, S, H, U):
+    B, D = 2, 64
+    q, k, v = wl.make_qkv(B, H, S, D, dtype, 42)
+    so, ho = oracle.uneven_offsets(S, U), oracle.uneven_offsets(H, U)
+    fq, fk, fv = (_flat(t, so) for t in (q, k, v))
+    out, lse = cp.ulysses_anything_attention(fq.cuda(), fk.cuda(), fv.cuda(), B, H, D, so, ho)
+    torch.cuda.synchronize()
+    ro, rl = oracle.ulysses_anything_attention(_np(fq), _np(fk), _np(fv), B, H, D, so, ho)
+    tol_o, tol_l = TOL[dtype]
+    assert np.abs(_np(out) - ro).max() <= tol_o
+    assert np.abs(_np(lse) - rl).max() <= tol_l
+
+
 # ---------------------------------------------------------------- failure surfacing
 def test_bounded_wait_reports_timeout(cuda_ok):
     assert cp.last_device_error() == 0
