@@ -257,25 +257,61 @@ def run_cuda(args):
     kernel_ms = float(np.mean(times))          # one launch per step
     gpu_launches = args.steps                  # one cp_ring_attention kernel per step
 
-    # ---- end to end through the C-ABI with host buffers
+    # ---- end to end through the C-ABI with host buffers: every step copies
+    # its q/k/v from pinned host memory and reads its output and lse back.
+    # Steps are pipelined over two device buffer sets and three streams, so
+    # step i+1's upload, step i's attention and step i-1's download overlap
+    # (PCIe moves both directions at once).
     hq, hk, hv = (t.pin_memory() for t in (q, k, v))
     hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    sets = [(dq, dk, dv, out, lse)] + [tuple(torch.empty_like(t) for t in (dq, dk, dv, out, lse))]
+    s_up, s_comp, s_down = (torch.cuda.Stream(dev) for _ in range(3))
 
-    def e2e_step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        cp.ring_attention(dq, dk, dv, offs, out=out, lse=lse)
-        hout.copy_(out, non_blocking=True)
-        hlse.copy_(lse, non_blocking=True)
+    def e2e_run(n):
+        ev_in_free = [torch.cuda.Event() for _ in range(2)]    # attention done with set
+        ev_out_free = [torch.cuda.Event() for _ in range(2)]   # download done with set
+        for e in ev_in_free + ev_out_free:
+            e.record(torch.cuda.current_stream(dev))
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(s_up)
+        s_comp.wait_event(t0)
+        s_down.wait_event(t0)
+        for i in range(n):
+            a, bq, bk, bv, bo, bl = i % 2, *sets[i % 2]
+            s_up.wait_event(ev_in_free[a])
+            with torch.cuda.stream(s_up):
+                bq.copy_(hq, non_blocking=True)
+                bk.copy_(hk, non_blocking=True)
+                bv.copy_(hv, non_blocking=True)
+            up = torch.cuda.Event()
+            up.record(s_up)
+            s_comp.wait_event(up)
+            s_comp.wait_event(ev_out_free[a])
+            with torch.cuda.stream(s_comp):
+                cp.ring_attention(bq, bk, bv, offs, out=bo, lse=bl)
+            ev_in_free[a] = torch.cuda.Event()
+            ev_in_free[a].record(s_comp)
+            s_down.wait_event(ev_in_free[a])
+            with torch.cuda.stream(s_down):
+                hout.copy_(bo, non_blocking=True)
+                hlse.copy_(bl, non_blocking=True)
+            ev_out_free[a] = torch.cuda.Event()
+            ev_out_free[a].record(s_down)
+        s_down.wait_stream(s_up)
+        s_down.wait_stream(s_comp)
+        t1.record(s_down)
+        torch.cuda.synchronize(dev)
+        return t0.elapsed_time(t1) / n
 
     e2e_steps = max(3, min(args.steps, 30))
+    e2e_run(3)                                    # warm-up
     _barrier(pg, dev)
-    e2e_times = _time_loop(e2e_step, e2e_steps, 2, lambda: None, stream)
-    e2e_ms = _max_over_ranks(pg, float(np.mean(e2e_times)), dev)
+    e2e_ms = _max_over_ranks(pg, e2e_run(e2e_steps), dev)
     h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
     d2h = out.numel() * 4 + lse.numel() * 4
+    del sets
 
     peaks, peak_src = _peaks()
     tc_peak = float(peaks["bf16_tflops"])
@@ -371,7 +407,9 @@ def run_cuda(args):
                          "algorithmic": "4*D flops per (query, key, head): 2.609e11 per launch"},
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_ms},
+                    "ms_per_step": e2e_ms,
+                    "how": "pinned host q/k/v -> device, cp_ring_attention, out+lse -> "
+                           "pinned host, every step; steps pipelined on 3 streams"},
             "gpu_launches": gpu_launches,
             "clocks": sampler.summary(),
             "components": components,

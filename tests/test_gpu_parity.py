@@ -198,6 +198,30 @@ def test_fused_ring_matches_literal_walk(cuda_ok, dtype):
         assert (lacc - fl).abs().max().item() <= tol_l
 
 
+@pytest.mark.parametrize("B,H,Sq,Skv,D,out_dtype", [(3, 2, 300, 200, 128, torch.float32),
+                                                    (2, 5, 129, 640, 64, torch.bfloat16),
+                                                    (1, 1, 1000, 3, 128, torch.bfloat16)])
+def test_ring_tensor_core_shapes(cuda_ok, B, H, Sq, Skv, D, out_dtype):
+    """Batches, S_q != S_kv, a query view whose heads are strided (every other
+    head of a wider tensor), bf16 output, and no lse output."""
+    g = torch.Generator().manual_seed(B * 100 + H)
+    wide = torch.randn(B, Sq, 2 * H, D, generator=g).bfloat16()
+    q = wide[:, :, ::2]                       # head stride 2*D: TMA reads it in place
+    k = torch.randn(B, Skv, H, D, generator=g).bfloat16()
+    v = torch.randn(B, Skv, H, D, generator=g).bfloat16()
+    offs = wl.chunk_offsets(wl.ring_chunk_lengths(Skv, 3))
+    ro, rl = oracle.attention(_np(q), _np(k), _np(v))
+    dq = wide.cuda()[:, :, ::2]
+    assert not dq.is_contiguous()
+    out, lse = cp.ring_attention(dq, k.cuda(), v.cuda(), offs, out_dtype=out_dtype)
+    out2, none = cp.ring_attention(dq, k.cuda(), v.cuda(), offs, out_dtype=out_dtype,
+                                   want_lse=False)
+    torch.cuda.synchronize()
+    assert none is None
+    _check(out, lse, ro, rl, torch.bfloat16)
+    assert torch.equal(out, out2)
+
+
 def test_constant_v_and_zero_q_closed_forms(cuda_ok):
     g = torch.Generator().manual_seed(18)
     S = 400
