@@ -344,6 +344,22 @@ def run_cuda(args):
         components[name] = {"shape": list(x.shape), "bytes": pbytes, "ms": float(np.mean(t_p)),
                             "GB/s": gbs, "frac_of_hbm": gbs / hbm_peak}
     del x, y, x2, oi, li, acc, lacc
+    # the literal ring walk on the FLUX workload: one launch per arriving K/V
+    # chunk, the first writing (out, lse), the others merging into them
+    kcs = [(dk[:, offs[c]:offs[c + 1]], dv[:, offs[c]:offs[c + 1]])
+           for c in range(w.ring_degree)]
+
+    def literal_ring():
+        cp.attn_partial(dq, *kcs[0], out=out, lse=lse)
+        for kc, vc in kcs[1:]:
+            cp.attn_partial_merge(dq, kc, vc, out, lse)
+
+    t_r = _time_loop(literal_ring, n_merge, 3, flush, stream)
+    tf = flops / (np.mean(t_r) * 1e-3) / 1e12
+    components["ring_per_chunk_partial_merge"] = {
+        "launches": w.ring_degree, "ms": float(np.mean(t_r)), "TFLOP/s": tf,
+        "frac_of_bf16_peak": tf / tc_peak,
+        "vs_single_launch": float(kernel_ms / np.mean(t_r))}
     # unified R=2 x U=2 grid (B=2, S=8192, H=24, D=128) from sequence shards
     uq, uk, uv = wl.make_workload_inputs(u)
     ush = [wl.sequence_shards(t, 4).to(dev) for t in (uq, uk, uv)]

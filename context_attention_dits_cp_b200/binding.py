@@ -28,7 +28,7 @@ STATUS = {
     -5: "CP_ERR_OFFSETS", -6: "CP_ERR_DEGREE", -7: "CP_ERR_CUDA", -8: "CP_ERR_TIMEOUT",
     -9: "CP_ERR_WORKSPACE", -10: "CP_ERR_ALIAS",
 }
-EXPORTS = ("cp_attn_partial", "cp_lse_merge", "cp_ring_attention", "cp_ulysses_permute",
+EXPORTS = ("cp_attn_partial", "cp_attn_partial_merge", "cp_lse_merge", "cp_ring_attention", "cp_ulysses_permute",
            "cp_usp_attention", "cp_usp_attention_static", "cp_usp_workspace_bytes",
            "cp_ulysses_anything_permute", "cp_ulysses_anything_attention",
            "cp_ulysses_anything_workspace_bytes", "cp_ring_chunk_offsets",
@@ -62,6 +62,7 @@ def lib() -> ctypes.CDLL:
         P = ctypes.POINTER(CpTensor)
         vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
         L.cp_attn_partial.argtypes = [P, P, P, f32, P, P, vp]
+        L.cp_attn_partial_merge.argtypes = [P, P, P, f32, P, P, vp]
         L.cp_lse_merge.argtypes = [P, P, P, P, vp]
         L.cp_ring_attention.argtypes = [P, P, P, ctypes.POINTER(i64), i32, f32, P, P, vp]
         L.cp_ulysses_permute.argtypes = [P, P, i32, i32, vp]
@@ -139,6 +140,15 @@ def attn_partial(q, k_chunk, v_chunk, scale=None, out=None, lse=None, out_dtype=
     _check(lib().cp_attn_partial(_ref(dq), _ref(dk), _ref(dv), _scale(scale), _ref(do),
                                  _ref(dl), _stream(q.device)), "cp_attn_partial")
     return out, lse
+
+
+def attn_partial_merge(q, k_chunk, v_chunk, out_acc, lse_acc, scale=None):
+    """One ring step folded into the fp32 accumulator in place
+    (cp_attn_partial_merge)."""
+    dq, dk, dv, do, dl = desc(q), desc(k_chunk), desc(v_chunk), desc(out_acc), desc(lse_acc)
+    _check(lib().cp_attn_partial_merge(_ref(dq), _ref(dk), _ref(dv), _scale(scale), _ref(do),
+                                       _ref(dl), _stream(q.device)), "cp_attn_partial_merge")
+    return out_acc, lse_acc
 
 
 def lse_merge(out_acc, lse_acc, out_i, lse_i):

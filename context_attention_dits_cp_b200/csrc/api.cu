@@ -192,6 +192,21 @@ int cp_attn_partial(const cp_tensor* q, const cp_tensor* k_chunk, const cp_tenso
   return run_attention(a, as_stream(stream));
 }
 
+int cp_attn_partial_merge(const cp_tensor* q, const cp_tensor* k_chunk,
+                          const cp_tensor* v_chunk, float scale, cp_tensor* out_acc,
+                          cp_tensor* lse_acc, void* stream) {
+  RingArgs a;
+  int st = prepare_attention(q, k_chunk, v_chunk, scale, out_acc, lse_acc, false, &a);
+  if (st) return st;
+  if (out_acc->dtype != CP_F32) return CP_ERR_DTYPE;   // the accumulator is fp32
+  if (k_chunk->shape[1] == 0) return CP_OK;           // an empty chunk merges as identity
+  const int64_t offs[2] = {0, k_chunk->shape[1]};
+  a.chunk_off = offs;
+  a.n_chunks = 1;
+  a.merge = true;
+  return run_attention(a, as_stream(stream));
+}
+
 int cp_ring_attention(const cp_tensor* q, const cp_tensor* k, const cp_tensor* v,
                       const int64_t* chunk_offsets, int n_chunks, float scale, cp_tensor* out,
                       cp_tensor* lse, void* stream) {

@@ -34,6 +34,7 @@ struct F32Params {
   long long v_sb, v_ss, v_sh;
   void* out;
   int out_bf16;
+  int merge;
   long long o_sb, o_ss, o_sh;
   float* lse;
   long long l_sb, l_sh, l_ss;
@@ -123,18 +124,35 @@ __global__ void __launch_bounds__(128) attn_ring_f32_kernel(const __grid_constan
   for (int r = 0; r < kRowsPerWarp; ++r) {
     const int s = r0 + warp * kRowsPerWarp + r;
     if (s >= p.S_q) continue;
-    const float inv_l = 1.f / l[r];
+    float o_w = 1.f / l[r];
+    const float lse_c = m[r] + logf(l[r]);
     const long long base = b * p.o_sb + (long long)s * p.o_ss + h * p.o_sh;
+    float* lse_p = p.lse != nullptr ? p.lse + b * p.l_sb + h * p.l_sh + (long long)s * p.l_ss
+                                    : nullptr;
+    if (p.merge) {
+      // fp32 log-sum-exp merge with the accumulator already in (out, lse)
+      const float a = *lse_p;
+      const float nl = a == -INFINITY ? lse_c
+                                      : fmaxf(a, lse_c) + log1pf(expf(-fabsf(a - lse_c)));
+      const float acc_w = a == -INFINITY ? 0.f : expf(a - nl);
+      o_w *= expf(lse_c - nl);
+      float* o = reinterpret_cast<float*>(p.out);
+#pragma unroll
+      for (int i = 0; i < NV; ++i)
+        o[base + lane + 32 * i] = fmaf(acc_w, o[base + lane + 32 * i], acc[r][i] * o_w);
+      __syncwarp();
+      if (lane == 0) *lse_p = nl;
+      continue;
+    }
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
-      const float o = acc[r][i] * inv_l;
+      const float o = acc[r][i] * o_w;
       if (p.out_bf16)
         reinterpret_cast<__nv_bfloat16*>(p.out)[base + lane + 32 * i] = __float2bfloat16_rn(o);
       else
         reinterpret_cast<float*>(p.out)[base + lane + 32 * i] = o;
     }
-    if (lane == 0 && p.lse != nullptr)
-      p.lse[b * p.l_sb + h * p.l_sh + (long long)s * p.l_ss] = m[r] + logf(l[r]);
+    if (lane == 0 && lse_p != nullptr) *lse_p = lse_c;
   }
 }
 
@@ -179,6 +197,7 @@ int launch_attn_ring_f32(const RingArgs& a, cudaStream_t stream) {
   prm.v_sh = a.v.stride[2];
   prm.out = a.out.data;
   prm.out_bf16 = a.out.dtype == CP_BF16;
+  prm.merge = a.merge ? 1 : 0;
   prm.o_sb = a.out.stride[0];
   prm.o_ss = a.out.stride[1];
   prm.o_sh = a.out.stride[2];

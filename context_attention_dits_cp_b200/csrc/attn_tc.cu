@@ -90,6 +90,7 @@ struct AttnTcParams {
   int* err;
   long long l_sb, l_sh, l_ss;    // lse strides (elements)
   int out_bf16;
+  int merge;                     // fold this result into (out, lse) instead of overwriting
   int B, H, S_q, S_kv;
   int seg_q, seg_kv;             // tokens per segment (S itself for one segment)
   int n_q_blocks;                // ceil(S_q / 256)
@@ -149,7 +150,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* o_done = p_ready + 2;       // [2]
   uint64_t* epi_full = o_done + 2;      // [2] a round of staged output is in smem
   uint64_t* epi_free = epi_full + 2;    // [2] TMA has read the staged round
-  uint64_t* drain = epi_free + 2;       // [1]
+  uint64_t* acc_full = epi_free + 2;    // [2] merge mode: the accumulator round is in smem
+  uint64_t* drain = acc_full + 2;       // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -174,6 +176,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&o_done[t], 1);
       mbar_init(&epi_full[t], kBlockM / 32);   // one arrive per softmax warp
       mbar_init(&epi_free[t], 1);
+      mbar_init(&acc_full[t], 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -404,10 +407,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // the staging buffer to the storing thread and back through bounded
       // mbarrier waits, so a warp that gave up never blocks the others.
       const int s_row = q0 + t * kBlockM + row;
-      const float inv_l = 1.0f / l_run;
-      if (p.lse != nullptr && s_row < p.S_q)
-        p.lse[b * p.l_sb + h * p.l_sh + (long long)s_row * p.l_ss] =
-            (m_run + log2f(l_run)) * 0.69314718055994530942f;
+      const float lse_c = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+      float o_w = 1.0f / l_run;   // weight of the raw accumulator O
+      float acc_w = 0.f;          // merge mode: weight of the (out, lse) already there
+      float* lse_p = p.lse != nullptr && s_row < p.S_q
+                         ? p.lse + b * p.l_sb + h * p.l_sh + (long long)s_row * p.l_ss
+                         : nullptr;
+      if (p.merge) {
+        // fp32 log-sum-exp merge with the accumulator (ContextParallelConfig
+        // .convert_to_fp32): lse' = max + log1p(exp(-|a - b|))
+        const float a = lse_p ? *lse_p : -INFINITY;
+        const float mx = fmaxf(a, lse_c);
+        const float nl = a == -INFINITY ? lse_c : mx + log1pf(expf(-fabsf(a - lse_c)));
+        acc_w = a == -INFINITY ? 0.f : expf(a - nl);
+        o_w *= expf(lse_c - nl);
+        if (lse_p) *lse_p = nl;
+      } else if (lse_p) {
+        *lse_p = lse_c;
+      }
+      const float inv_l = o_w;
       uint8_t* stage = sQ + t * L::kTileBytes;
       const int esz = p.out_bf16 ? 2 : 4;
       const int cols_per_box = 128 / esz;               // 32 fp32 or 64 bf16
@@ -418,10 +436,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // the previous round's TMA stores must have read the staging buffer
         if (rounds > 0 && !(ok = mbar_wait(&epi_free[t], (rounds - 1) & 1, abort_flag, p.err)))
           break;
+        const int r0 = q0 + t * kBlockM;
+        if (p.merge) {
+          // bring this round's accumulator boxes into the staging buffer
+          if (leader) {
+            mbar_arrive_expect_tx(&acc_full[t], boxes_per_round * (128 * 128));
+            for (int bx = b0; bx < b0 + boxes_per_round; ++bx)
+              tma_load_5d(stage + (bx - b0) * (128 * 128), &p.tmap_out, &acc_full[t],
+                          bx * cols_per_box, r0 % p.seg_q, h, r0 / p.seg_q, b);
+          }
+          if (!(ok = mbar_wait(&acc_full[t], rounds & 1, abort_flag, p.err))) break;
+        }
         for (int bx = b0; bx < b0 + boxes_per_round; ++bx) {
           uint8_t* box = stage + (bx - b0) * (128 * 128) + row * 128;
           // this box holds O columns [bx * cols_per_box, (bx+1) * cols_per_box)
-          if (p.out_bf16) {
+          if (p.merge) {          // fp32 accumulator: out' = acc_w * out + o_w * O
+            float o[32];
+            tmem_ld32(tO + bx * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              float4* cell = reinterpret_cast<float4*>(box + ((k ^ (row & 7)) << 4));
+              const float4 a4 = *cell;
+              *cell = make_float4(fmaf(acc_w, a4.x, o[4 * k] * inv_l),
+                                  fmaf(acc_w, a4.y, o[4 * k + 1] * inv_l),
+                                  fmaf(acc_w, a4.z, o[4 * k + 2] * inv_l),
+                                  fmaf(acc_w, a4.w, o[4 * k + 3] * inv_l));
+            }
+          } else if (p.out_bf16) {
 #pragma unroll
             for (int hlf = 0; hlf < 2; ++hlf) {
               float o[32];
@@ -454,7 +496,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) mbar_arrive(&epi_full[t]);
         if (leader) {
           if (!(ok = mbar_wait(&epi_full[t], rounds & 1, abort_flag, p.err))) break;
-          const int r0 = q0 + t * kBlockM;
           for (int bx = b0; bx < b0 + boxes_per_round; ++bx)
             tma_store_5d(&p.tmap_out, stage + (bx - b0) * (128 * 128), bx * cols_per_box,
                          r0 % p.seg_q, h, r0 / p.seg_q, b);
@@ -572,6 +613,7 @@ int launch_attn_ring_tc(const RingArgs& a, cudaStream_t stream) {
   if ((st = encode_out(&prm.tmap_out, a.out)) != CP_OK) return st;
   prm.out = a.out.data;
   prm.out_bf16 = a.out.dtype == CP_BF16;
+  prm.merge = a.merge ? 1 : 0;
   prm.lse = static_cast<float*>(a.lse.data);
   prm.l_sb = a.lse.stride[0];
   prm.l_sh = a.lse.stride[1];

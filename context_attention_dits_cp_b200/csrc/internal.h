@@ -40,6 +40,7 @@ struct RingArgs {
   const int64_t* chunk_off = nullptr;   // host, n_chunks + 1
   int n_chunks = 0;
   float scale = 0.f;
+  bool merge = false;      // fold into (out, lse) with the fp32 LSE merge
   int* dev_err = nullptr;
 };
 

@@ -97,6 +97,20 @@ int cp_attn_partial(const cp_tensor* q, const cp_tensor* k_chunk,
                     cp_tensor* lse, void* stream);
 
 /*
+ * cp_attn_partial_merge -- one ring step with the merge fused into its
+ * epilogue: the partial of q against this K/V chunk is folded into the fp32
+ * accumulator (out_acc, lse_acc) in place, with the same log-sum-exp merge
+ * as cp_lse_merge.  This is the call a ring rank makes as each chunk
+ * arrives; it writes no separate partial and needs no merge pass.
+ *   out_acc [B, S_q, H, D] f32 (in/out)   lse_acc [B, H, S_q] f32 (in/out)
+ * Start from (0, -inf).  An empty chunk leaves the accumulator unchanged.
+ */
+int cp_attn_partial_merge(const cp_tensor* q, const cp_tensor* k_chunk,
+                          const cp_tensor* v_chunk, float scale,
+                          cp_tensor* out_acc, cp_tensor* lse_acc,
+                          void* stream);
+
+/*
  * cp_lse_merge -- fold one partial into an fp32 accumulator, in place
  * (ContextParallelConfig.convert_to_fp32).  Per row, with a = lse_acc and
  * b = lse_i:

@@ -85,6 +85,15 @@ def test_attn_partial_argument_errors():
     assert _partial(q, k, v, alias, lse) == -10
 
 
+def test_partial_merge_errors():
+    q, k, v, out, lse = _ok_args()
+    L = bd.lib()
+    r = ctypes.byref
+    bf_out = _t([1, 256, 2, 128], bd.CP_BF16, FAKE + (3 << 24))
+    assert L.cp_attn_partial_merge(r(q), r(k), r(v), 0.0, r(bf_out), r(lse), None) == -2
+    assert L.cp_attn_partial_merge(r(q), r(k), r(v), 0.0, r(out), None, None) == -1
+
+
 def test_ring_offsets_errors():
     q, k, v, out, lse = _ok_args()
     L = bd.lib()

@@ -222,6 +222,33 @@ def test_ring_tensor_core_shapes(cuda_ok, B, H, Sq, Skv, D, out_dtype):
     assert torch.equal(out, out2)
 
 
+@pytest.mark.parametrize("dtype,D", [(torch.bfloat16, 128), (torch.bfloat16, 64),
+                                     (torch.float32, 128)])
+def test_partial_merge_walk_equals_oneshot_and_literal(cuda_ok, dtype, D):
+    """A ring walk made only of cp_attn_partial_merge calls (chunks arriving
+    in ring order from rank 1, with an empty chunk) equals one-shot attention
+    and the partial + standalone-merge walk."""
+    B, H, Sq, Skv = 2, 3, 333, 700
+    q, k, v = wl.make_qkv(B, H, Sq, D, dtype, 43, S_kv=Skv)
+    dq, dk, dv = _dev(q, k, v)
+    offs = [0, 250, 250, 500, 700]
+    acc = torch.zeros(B, Sq, H, D, device="cuda")
+    lacc = torch.full((B, H, Sq), -float("inf"), device="cuda")
+    lit = acc.clone()
+    llit = lacc.clone()
+    for c in (1, 2, 3, 0):
+        kc, vc = dk[:, offs[c]:offs[c + 1]], dv[:, offs[c]:offs[c + 1]]
+        cp.attn_partial_merge(dq, kc, vc, acc, lacc)
+        oc, lc = cp.attn_partial(dq, kc, vc)
+        cp.lse_merge(lit, llit, oc, lc)
+    torch.cuda.synchronize()
+    ro, rl = oracle.attention(_np(q), _np(k), _np(v))
+    _check(acc, lacc, ro, rl, dtype)
+    tol_o, tol_l = TOL[dtype]
+    assert (acc - lit).abs().max().item() <= tol_o
+    assert (lacc - llit).abs().max().item() <= tol_l
+
+
 def test_constant_v_and_zero_q_closed_forms(cuda_ok):
     g = torch.Generator().manual_seed(18)
     S = 400
