@@ -56,13 +56,6 @@ constexpr int kBlockN = 128;    // keys per tile
 #define CP_RESCALE_LOG2_THRESHOLD 8
 #endif
 constexpr float kRescaleThreshold = (float)CP_RESCALE_LOG2_THRESHOLD;
-// Of every 8 consecutive column pairs of a full key tile, this many take
-// their exponentials from the FMA-pipe polynomial (exp2_fma) and the rest
-// from the MUFU unit.
-#ifndef CP_EXP2_FMA_PAIRS_PER_8
-#define CP_EXP2_FMA_PAIRS_PER_8 0
-#endif
-constexpr int kExp2FmaPairsPer8 = CP_EXP2_FMA_PAIRS_PER_8;
 // K/V ring slots (one 128-key tile of K or V each).  Each K/V tile feeds
 // two query tiles, so a slot stays busy for most of an iteration; the ring
 // must be deep enough that the next K tile is already resident when the
@@ -346,8 +339,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
       {
         // Rescale the rows whose max moved beyond the threshold, then
-        // exponentiate.  Tiles cut by their chunk's end use the MUFU unit
-        // only, which maps the masked -inf columns to exactly 0.
+        // exponentiate on the MUFU unit, which maps the masked -inf columns
+        // of a tile cut by its chunk's end to exactly 0.
         const bool need = m_tile > m_run + kRescaleThreshold;
         if (__any_sync(0xffffffffu, need)) {
           const float alpha = need ? ex2_approx(m_run - m_tile) : 1.0f;
@@ -376,14 +369,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int i = 0; i < 16; ++i) {
             const int e = c * 32 + 2 * i;
             const float2 x = fma2(make_float2(s[e], s[e + 1]), sl2x2, nmx2);
-            float2 pp;
-            if (valid == kBlockN && (i & 7) < kExp2FmaPairsPer8) {
-              pp.x = exp2_fma(x.x);
-              pp.y = exp2_fma(x.y);
-            } else {
-              pp.x = ex2_approx(x.x);
-              pp.y = ex2_approx(x.y);
-            }
+            const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
             acc[i & 3] = add2(acc[i & 3], pp);
             pk[i] = pack_bf16x2(pp.x, pp.y);
           }

@@ -308,25 +308,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for x <= 8 (larger x is never produced by the
-// softmax).  Cody-Waite style split x = n + f, n = round(x), f in [-1/2, 1/2]:
-// adding 1.5 * 2^23 leaves round(x) in the low mantissa bits of y, so
-// bits(y) << 23 is n << 23 (mod 2^32) and adding it to bits(p(f)) scales
-// p(f) by 2^n.  p is the degree-3 minimax approximation of 2^f in relative
-// error on [-1/2, 1/2] (fit_exp2_poly.py, Remez exchange; max relative error
-// 7.5e-5 with these float32 coefficients, far below the bf16 rounding of P).
-// x is clamped at -125 so 2^n stays a normal float; -inf gives ~2^-125.
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -125.0f);
-  const float y = x + 12582912.0f;
-  const float n = y - 12582912.0f;
-  const float f = x - n;
-  float p = fmaf(5.517166853e-02f, f, 2.426111251e-01f);
-  p = fmaf(p, f, 6.932609677e-01f);
-  p = fmaf(p, f, 9.999280572e-01f);
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(y) << 23));
-}
-
 // Packed fp32 pairs (sm_100 f32x2 instructions): one instruction updates
 // two independent lanes of data.
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
