@@ -65,6 +65,29 @@ int check_basic(const cp_tensor* t, int ndim) {
   return CP_OK;
 }
 
+// An output must not map two of its elements to one address (a zero stride,
+// or dims that interleave): the kernels would race on it.  Sufficient test:
+// with the dims of extent > 1 ordered by stride, each stride is at least the
+// span of the dims below it.
+bool self_overlapping(const cp_tensor* t) {
+  int64_t st[CP_MAX_DIMS], sh[CP_MAX_DIMS];
+  int n = 0;
+  for (int i = 0; i < t->ndim; ++i) {
+    if (t->shape[i] <= 1) continue;
+    if (t->stride[i] == 0) return true;
+    int j = n++;
+    for (; j > 0 && st[j - 1] > t->stride[i]; --j) {
+      st[j] = st[j - 1];
+      sh[j] = sh[j - 1];
+    }
+    st[j] = t->stride[i];
+    sh[j] = t->shape[i];
+  }
+  for (int k = 0; k + 1 < n; ++k)
+    if (st[k + 1] < st[k] * sh[k]) return true;
+  return false;
+}
+
 // Element-stride / base alignment to `bytes` for every dim but the last,
 // which must be contiguous.
 int check_vector_layout(const cp_tensor* t, int bytes) {
@@ -111,6 +134,7 @@ int prepare_attention(const cp_tensor* q, const cp_tensor* k, const cp_tensor* v
     if (lse->dtype != CP_F32) return CP_ERR_DTYPE;
   }
   if (q->dtype != k->dtype || q->dtype != v->dtype) return CP_ERR_DTYPE;
+  if (self_overlapping(out) || (lse && self_overlapping(lse))) return CP_ERR_ALIAS;
   const int64_t B = q->shape[0], Sq = q->shape[1], H = q->shape[2], D = q->shape[3];
   const int64_t Skv = k->shape[1];
   if (D != 64 && D != 128) return CP_ERR_SHAPE;
@@ -241,6 +265,7 @@ int cp_lse_merge(cp_tensor* out_acc, cp_tensor* lse_acc, const cp_tensor* out_i,
         reinterpret_cast<uintptr_t>(lse_i->data) % 4)
       return CP_ERR_ALIGN;
   }
+  if (self_overlapping(out_acc) || self_overlapping(lse_acc)) return CP_ERR_ALIAS;
   const TensorView va = view_of(out_acc), vla = view_of(lse_acc), vi = view_of(out_i),
                    vli = view_of(lse_i);
   if (overlaps(va, vi) || overlaps(va, vla) || overlaps(va, vli) || overlaps(vla, vi) ||
@@ -274,7 +299,7 @@ int cp_ulysses_permute(const cp_tensor* x, cp_tensor* y, int degree, int dir, vo
     if (t->shape[3] > 1 && t->stride[3] != D) return CP_ERR_ALIGN;
   }
   const TensorView vx = view_of(x), vy = view_of(y);
-  if (overlaps(vx, vy)) return CP_ERR_ALIAS;
+  if (self_overlapping(y) || overlaps(vx, vy)) return CP_ERR_ALIAS;
   return launch_ulysses_permute(vx, vy, degree, dir, as_stream(stream));
 }
 
@@ -313,6 +338,7 @@ int cp_usp_attention(const cp_tensor* qs, const cp_tensor* ks, const cp_tensor* 
     if (lse->shape[0] != B || lse->shape[1] != H || lse->shape[2] != S) return CP_ERR_SHAPE;
   }
   if (R > CP_MAX_CHUNKS) return CP_ERR_DEGREE;
+  if (self_overlapping(outs) || (lse && self_overlapping(lse))) return CP_ERR_ALIAS;
   if (B == 0 || S == 0 || H == 0) return CP_OK;
 
   // Fused: attention reads q/k/v and writes out in the shard layout through
@@ -514,6 +540,7 @@ int cp_ulysses_anything_attention(const cp_tensor* q, const cp_tensor* k, const 
     if ((st = check_basic(lse, 3))) return st;
     if (lse->dtype != CP_F32) return CP_ERR_DTYPE;
     if (lse->shape[0] != B || lse->shape[1] != H || lse->shape[2] != S) return CP_ERR_SHAPE;
+    if (self_overlapping(lse)) return CP_ERR_ALIAS;
   }
   const TensorView vo = view_of(out);
   if (overlaps(vo, view_of(q)) || overlaps(vo, view_of(k)) || overlaps(vo, view_of(v)))

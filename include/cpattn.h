@@ -80,7 +80,9 @@ enum {
   CP_ERR_CUDA = -7,      /* a CUDA runtime/driver call failed               */
   CP_ERR_TIMEOUT = -8,   /* a bounded device-side wait gave up              */
   CP_ERR_WORKSPACE = -9, /* workspace missing or too small                  */
-  CP_ERR_ALIAS = -10     /* an output overlaps an input it must not alias   */
+  CP_ERR_ALIAS = -10     /* an output overlaps an input it must not alias,
+                            or maps two of its own elements to one address
+                            (a zero stride, or dims that interleave)        */
 };
 
 /*

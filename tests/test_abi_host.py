@@ -85,6 +85,28 @@ def test_attn_partial_argument_errors():
     assert _partial(q, k, v, alias, lse) == -10
 
 
+def test_self_overlapping_outputs_are_rejected():
+    """An output that maps two elements to one address (a broadcast dim, or
+    dims that interleave) is refused before any launch."""
+    q, k, v, out, lse = _ok_args()
+    L = bd.lib()
+    r = ctypes.byref
+    bcast = _t([1, 256, 2, 128], bd.CP_F32, FAKE + (3 << 24), strides=[0, 0, 128, 1])
+    assert L.cp_attn_partial(r(q), r(k), r(v), 0.0, r(bcast), r(lse), None) == -10
+    interleaved = _t([1, 256, 2, 128], bd.CP_F32, FAKE + (3 << 24),
+                     strides=[256 * 2 * 128, 64, 128, 1])
+    assert L.cp_ring_attention(r(q), r(k), r(v), (ctypes.c_int64 * 2)(0, 300), 1, 0.0,
+                               r(interleaved), r(lse), None) == -10
+    lse_b = _t([1, 2, 256], bd.CP_F32, FAKE + (5 << 24), strides=[512, 0, 1])
+    assert L.cp_attn_partial(r(q), r(k), r(v), 0.0, r(out), r(lse_b), None) == -10
+    lse2 = _t([1, 2, 256], bd.CP_F32, FAKE + (6 << 24))
+    assert L.cp_lse_merge(r(bcast), r(lse), r(out), r(lse2), None) == -10
+    assert L.cp_lse_merge(r(out), r(lse), r(out), r(lse2), None) == -10   # plain alias
+    x = _t([2, 1, 8, 4, 128], bd.CP_BF16, FAKE)
+    y = _t([2, 1, 16, 2, 128], bd.CP_BF16, FAKE + (3 << 24), strides=[0, 4096, 256, 128, 1])
+    assert L.cp_ulysses_permute(r(x), r(y), 2, 0, None) == -10
+
+
 def test_partial_merge_errors():
     q, k, v, out, lse = _ok_args()
     L = bd.lib()

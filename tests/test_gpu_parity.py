@@ -249,6 +249,28 @@ def test_partial_merge_walk_equals_oneshot_and_literal(cuda_ok, dtype, D):
     assert (lacc - llit).abs().max().item() <= tol_l
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_partial_merge_into_strided_views(cuda_ok, dtype):
+    """The accumulator may be a view: every other head of a wider output and
+    an LSE whose rows are padded.  Entries outside the views stay untouched."""
+    B, H, Sq, Skv, D = 1, 2, 300, 384, 128
+    q, k, v = wl.make_qkv(B, H, Sq, D, dtype, 47, S_kv=Skv)
+    dq, dk, dv = _dev(q, k, v)
+    big = torch.full((B, Sq, 2 * H, D), 7.0, device="cuda")
+    acc = big[:, :, ::2]
+    acc.zero_()
+    lbig = torch.full((B, H, Sq + 20), 3.0, device="cuda")
+    lacc = lbig[:, :, 10:10 + Sq]
+    lacc.fill_(-float("inf"))
+    for lo, hi in ((256, 384), (0, 256)):
+        cp.attn_partial_merge(dq, dk[:, lo:hi], dv[:, lo:hi], acc, lacc)
+    torch.cuda.synchronize()
+    ro, rl = oracle.attention(_np(q), _np(k), _np(v))
+    _check(acc, lacc, ro, rl, dtype)
+    assert bool((big[:, :, 1::2] == 7.0).all())
+    assert bool((lbig[:, :, :10] == 3.0).all()) and bool((lbig[:, :, 10 + Sq:] == 3.0).all())
+
+
 def test_constant_v_and_zero_q_closed_forms(cuda_ok):
     g = torch.Generator().manual_seed(18)
     S = 400
