@@ -195,6 +195,17 @@ def _time_loop(fn, steps, warmup, flush, stream):
 
 
 # ---------------------------------------------------------------- CUDA arm
+def workload_config(w):
+    """The benchmark line's `config`, shared by both arms."""
+    from context_attention_dits_cp_b200 import workloads as wl
+    lens = wl.ring_chunk_lengths(w.S, w.ring_degree)
+    return {"workload": WORKLOAD, "B": w.B, "H": w.H, "S": w.S, "D": w.D,
+            "ring_degree": w.ring_degree, "chunks": [int(c) for c in lens],
+            "inputs": "N(0,1) q/k/v, key tokens scaled by U[0.5,2]",
+            "out": "fp32 out + fp32 lse", "l2": "flushed between steps",
+            "per_gpu": "independent replica per GPU"}
+
+
 def run_cuda(args):
     import context_attention_dits_cp_b200 as cp
     from context_attention_dits_cp_b200 import workloads as wl
@@ -409,12 +420,7 @@ def run_cuda(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "S": w.S, "D": w.D,
-                       "ring_degree": w.ring_degree, "chunks": [offs[i + 1] - offs[i]
-                                                                for i in range(w.ring_degree)],
-                       "inputs": "N(0,1) q/k/v, key tokens scaled by U[0.5,2]",
-                       "out": "fp32 out + fp32 lse", "l2": "flushed between steps",
-                       "per_gpu": "independent replica per GPU"},
+            "config": workload_config(w),
             "pct_of_bf16_peak": 100.0 * value / (world * tc_peak),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": tc_peak,
                          "unit": "TFLOP/s", "frac": achieved / tc_peak, "traffic": traffic,
@@ -528,8 +534,7 @@ def run_reference(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "S": w.S, "D": w.D,
-                   "ring_degree": w.ring_degree},
+        "config": workload_config(w),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": f"{rows} random query rows x all {w.H} heads per step "
                                    f"against all {w.S} keys, fp64"},
