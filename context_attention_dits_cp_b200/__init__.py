@@ -6,7 +6,8 @@ composition, all running in the hand-written CUDA kernels of libcpattn.so
 (C-ABI in include/cpattn.h).  This package is the thin Python binding.
 """
 from .binding import (  # noqa: F401
-    CpError, attn_partial, attn_partial_merge, lse_merge, ring_attention, ring_chunk_offsets, ulysses_permute,
+    CpError, attn_partial, attn_partial_merge, lse_merge, ring_attention, ring_attention_gathered,
+    ring_chunk_offsets, ulysses_permute,
     usp_attention, usp_workspace_bytes, last_device_error, selftest_wait_timeout,
     ulysses_anything_permute, ulysses_anything_attention,
     attention_flops, SEQ_TO_HEAD, HEAD_TO_SEQ,

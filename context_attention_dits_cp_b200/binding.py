@@ -28,7 +28,7 @@ STATUS = {
     -5: "CP_ERR_OFFSETS", -6: "CP_ERR_DEGREE", -7: "CP_ERR_CUDA", -8: "CP_ERR_TIMEOUT",
     -9: "CP_ERR_WORKSPACE", -10: "CP_ERR_ALIAS",
 }
-EXPORTS = ("cp_attn_partial", "cp_attn_partial_merge", "cp_lse_merge", "cp_ring_attention", "cp_ulysses_permute",
+EXPORTS = ("cp_attn_partial", "cp_attn_partial_merge", "cp_lse_merge", "cp_ring_attention_gathered", "cp_ring_attention", "cp_ulysses_permute",
            "cp_usp_attention", "cp_usp_attention_static", "cp_usp_workspace_bytes",
            "cp_ulysses_anything_permute", "cp_ulysses_anything_attention",
            "cp_ulysses_anything_workspace_bytes", "cp_ring_chunk_offsets",
@@ -65,6 +65,8 @@ def lib() -> ctypes.CDLL:
         L.cp_attn_partial_merge.argtypes = [P, P, P, f32, P, P, vp]
         L.cp_lse_merge.argtypes = [P, P, P, P, vp]
         L.cp_ring_attention.argtypes = [P, P, P, ctypes.POINTER(i64), i32, f32, P, P, vp]
+        L.cp_ring_attention_gathered.argtypes = [P, P, P, ctypes.POINTER(i64), i32, i32, f32,
+                                                 i32, P, P, vp]
         L.cp_ulysses_permute.argtypes = [P, P, i32, i32, vp]
         L.cp_usp_attention.argtypes = [P, P, P, i32, i32, f32, vp, ctypes.c_size_t, P, P, vp]
         L.cp_usp_attention_static.argtypes = [P, P, P, i32, i32, f32, P, P, vp]
@@ -178,6 +180,28 @@ def ring_attention(q, k, v, chunk_offsets: Sequence[int], scale=None, out=None, 
     _check(lib().cp_ring_attention(_ref(dq), _ref(dk), _ref(dv), offs, len(chunk_offsets) - 1,
                                    _scale(scale), _ref(do), _ref(dl), _stream(q.device)),
            "cp_ring_attention")
+    return out, lse
+
+
+def ring_attention_gathered(q, k_gathered, v_gathered, chunk_lengths: Sequence[int],
+                            skip_chunk: int = -1, scale=None, out=None, lse=None,
+                            accumulate=False, out_dtype=torch.float32, want_lse=True):
+    """The ring over the slots [R, B, L, H, D] of a padded K/V all-gather;
+    chunk c is rows [0, chunk_lengths[c]) of slot c (cp_ring_attention_gathered).
+    With accumulate=True, (out, lse) is an fp32 accumulator updated in place."""
+    B, S, H, D = q.shape
+    if accumulate and (out is None or lse is None):
+        raise ValueError("accumulate=True needs the accumulator (out, lse)")
+    out = torch.empty((B, S, H, D), dtype=out_dtype, device=q.device) if out is None else out
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    lens = (ctypes.c_int64 * len(chunk_lengths))(*[int(x) for x in chunk_lengths])
+    dq, dk, dv, do, dl = desc(q), desc(k_gathered), desc(v_gathered), desc(out), desc(lse)
+    _check(lib().cp_ring_attention_gathered(_ref(dq), _ref(dk), _ref(dv), lens,
+                                            len(chunk_lengths), int(skip_chunk), _scale(scale),
+                                            1 if accumulate else 0, _ref(do), _ref(dl),
+                                            _stream(q.device)),
+           "cp_ring_attention_gathered")
     return out, lse
 
 

@@ -122,12 +122,14 @@ size_t usp_unfused_bytes(int64_t B, int64_t S, int64_t H, int64_t D, int in_dtyp
 
 // Shared validation of attention arguments.  On success fills `a` (without
 // chunk offsets) and reports whether there is anything to compute.
+// K/V are [B, S_kv, H, D], or with kv_ndim 5 the slots [G, B, L, H, D] of a
+// padded all-gather (token s = row s % L of slot s / L).
 int prepare_attention(const cp_tensor* q, const cp_tensor* k, const cp_tensor* v, float scale,
                       const cp_tensor* out, const cp_tensor* lse, bool lse_optional,
-                      RingArgs* a) {
+                      RingArgs* a, int kv_ndim = 4) {
   int st;
-  if ((st = check_basic(q, 4)) || (st = check_basic(k, 4)) || (st = check_basic(v, 4)) ||
-      (st = check_basic(out, 4)))
+  if ((st = check_basic(q, 4)) || (st = check_basic(k, kv_ndim)) ||
+      (st = check_basic(v, kv_ndim)) || (st = check_basic(out, 4)))
     return st;
   if (!lse_optional || lse) {
     if ((st = check_basic(lse, 3))) return st;
@@ -136,10 +138,10 @@ int prepare_attention(const cp_tensor* q, const cp_tensor* k, const cp_tensor* v
   if (q->dtype != k->dtype || q->dtype != v->dtype) return CP_ERR_DTYPE;
   if (self_overlapping(out) || (lse && self_overlapping(lse))) return CP_ERR_ALIAS;
   const int64_t B = q->shape[0], Sq = q->shape[1], H = q->shape[2], D = q->shape[3];
-  const int64_t Skv = k->shape[1];
   if (D != 64 && D != 128) return CP_ERR_SHAPE;
-  if (k->shape[0] != B || k->shape[2] != H || k->shape[3] != D) return CP_ERR_SHAPE;
-  for (int i = 0; i < 4; ++i)
+  const int kb = kv_ndim - 4;   // index of the batch dim of k / v
+  if (k->shape[kb] != B || k->shape[kb + 2] != H || k->shape[kb + 3] != D) return CP_ERR_SHAPE;
+  for (int i = 0; i < kv_ndim; ++i)
     if (v->shape[i] != k->shape[i]) return CP_ERR_SHAPE;
   for (int i = 0; i < 4; ++i)
     if (out->shape[i] != q->shape[i]) return CP_ERR_SHAPE;
@@ -176,8 +178,12 @@ int run_attention(RingArgs& a, cudaStream_t stream) {
   if (a.q.shape[1] == 0 || a.q.shape[0] == 0 || a.q.shape[2] == 0) return CP_OK;
   a.dev_err = device_error_ptr();
   if (!a.dev_err) return CP_ERR_CUDA;
-  const int64_t total = a.chunk_off[a.n_chunks] - a.chunk_off[0];
-  if (total == 0) return launch_fill_empty(a.out, a.lse, stream);
+  int64_t total = 0;
+  for (int c = 0; c < a.n_chunks; ++c) {
+    const int64_t len = (a.chunk_end ? a.chunk_end[c] : a.chunk_off[c + 1]) - a.chunk_off[c];
+    if (len > 0) total += len;
+  }
+  if (total == 0) return a.merge ? CP_OK : launch_fill_empty(a.out, a.lse, stream);
   if (a.q.dtype == CP_BF16) return launch_attn_ring_tc(a, stream);
   return launch_attn_ring_f32(a, stream);
 }
@@ -273,6 +279,34 @@ int cp_lse_merge(cp_tensor* out_acc, cp_tensor* lse_acc, const cp_tensor* out_i,
     return CP_ERR_ALIAS;
   if (B == 0 || S == 0 || H == 0) return CP_OK;
   return launch_lse_merge(va, vla, vi, vli, as_stream(stream));
+}
+
+int cp_ring_attention_gathered(const cp_tensor* q, const cp_tensor* k_gathered,
+                               const cp_tensor* v_gathered, const int64_t* chunk_lengths,
+                               int n_chunks, int skip_chunk, float scale, int accumulate,
+                               cp_tensor* out, cp_tensor* lse, void* stream) {
+  RingArgs a;
+  int st = prepare_attention(q, k_gathered, v_gathered, scale, out, lse, !accumulate, &a, 5);
+  if (st) return st;
+  if (accumulate && out->dtype != CP_F32) return CP_ERR_DTYPE;   // the accumulator is fp32
+  if (!chunk_lengths) return CP_ERR_NULL;
+  if (n_chunks < 1 || n_chunks > CP_MAX_CHUNKS || k_gathered->shape[0] != n_chunks)
+    return CP_ERR_OFFSETS;
+  if (skip_chunk < -1 || skip_chunk >= n_chunks) return CP_ERR_OFFSETS;
+  const int64_t L = k_gathered->shape[2];
+  if ((int64_t)n_chunks * L > 0x7fffffffLL) return CP_ERR_SHAPE;
+  int64_t starts[CP_MAX_CHUNKS + 1], ends[CP_MAX_CHUNKS];
+  for (int c = 0; c < n_chunks; ++c) {
+    if (chunk_lengths[c] < 0 || chunk_lengths[c] > L) return CP_ERR_OFFSETS;
+    starts[c] = c * L;
+    ends[c] = starts[c] + (c == skip_chunk ? 0 : chunk_lengths[c]);
+  }
+  starts[n_chunks] = n_chunks * L;
+  a.chunk_off = starts;
+  a.chunk_end = ends;
+  a.n_chunks = n_chunks;
+  a.merge = accumulate != 0;
+  return run_attention(a, as_stream(stream));
 }
 
 int cp_ulysses_permute(const cp_tensor* x, cp_tensor* y, int degree, int dir, void* stream) {

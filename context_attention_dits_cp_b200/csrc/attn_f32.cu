@@ -30,8 +30,10 @@ struct F32Params {
   const float* k;
   const float* v;
   long long q_sb, q_ss, q_sh;
-  long long k_sb, k_ss, k_sh;
-  long long v_sb, v_ss, v_sh;
+  // key token s is row s % seg_kv of slot s / seg_kv (one slot for [B, S, H, D])
+  long long k_sb, k_ss, k_sh, k_sg;
+  long long v_sb, v_ss, v_sh, v_sg;
+  int seg_kv;
   void* out;
   int out_bf16;
   int merge;
@@ -40,7 +42,8 @@ struct F32Params {
   long long l_sb, l_sh, l_ss;
   int B, H, S_q, n_row_blocks, n_chunks;
   float scale;
-  int chunk_off[CP_MAX_CHUNKS + 1];
+  int chunk_off[CP_MAX_CHUNKS + 1];   // chunk c covers key tokens [chunk_off[c], chunk_end[c])
+  int chunk_end[CP_MAX_CHUNKS];
 };
 
 __device__ __forceinline__ float warp_max(float x) {
@@ -83,15 +86,16 @@ __global__ void __launch_bounds__(128) attn_ring_f32_kernel(const __grid_constan
   }
 
   for (int c = 0; c < p.n_chunks; ++c) {
-    const int lo = p.chunk_off[c], hi = p.chunk_off[c + 1];
+    const int lo = p.chunk_off[c], hi = p.chunk_end[c];
     for (int t0 = lo; t0 < hi; t0 += kKeysPerTile) {
       const int n = min(kKeysPerTile, hi - t0);
       __syncthreads();   // everyone is done with the previous tile
       for (int i = threadIdx.x; i < n * D; i += blockDim.x) {
         const int j = i / D, d = i % D;
-        const long long key = t0 + j;
-        sK[j][d] = p.k[b * p.k_sb + key * p.k_ss + h * p.k_sh + d];
-        sV[j][d] = p.v[b * p.v_sb + key * p.v_ss + h * p.v_sh + d];
+        const int key = t0 + j;
+        const long long row = key % p.seg_kv, slot = key / p.seg_kv;
+        sK[j][d] = p.k[b * p.k_sb + row * p.k_ss + slot * p.k_sg + h * p.k_sh + d];
+        sV[j][d] = p.v[b * p.v_sb + row * p.v_ss + slot * p.v_sg + h * p.v_sh + d];
       }
       __syncthreads();
 #pragma unroll
@@ -189,12 +193,27 @@ int launch_attn_ring_f32(const RingArgs& a, cudaStream_t stream) {
   prm.q_sb = a.q.stride[0];
   prm.q_ss = a.q.stride[1];
   prm.q_sh = a.q.stride[2];
-  prm.k_sb = a.k.stride[0];
-  prm.k_ss = a.k.stride[1];
-  prm.k_sh = a.k.stride[2];
-  prm.v_sb = a.v.stride[0];
-  prm.v_ss = a.v.stride[1];
-  prm.v_sh = a.v.stride[2];
+  if (a.k.ndim == 5) {   // [G, B, L, H, D] slots
+    prm.k_sg = a.k.stride[0];
+    prm.k_sb = a.k.stride[1];
+    prm.k_ss = a.k.stride[2];
+    prm.k_sh = a.k.stride[3];
+    prm.v_sg = a.v.stride[0];
+    prm.v_sb = a.v.stride[1];
+    prm.v_ss = a.v.stride[2];
+    prm.v_sh = a.v.stride[3];
+    prm.seg_kv = (int)a.k.shape[2];
+  } else {
+    prm.k_sb = a.k.stride[0];
+    prm.k_ss = a.k.stride[1];
+    prm.k_sh = a.k.stride[2];
+    prm.v_sb = a.v.stride[0];
+    prm.v_ss = a.v.stride[1];
+    prm.v_sh = a.v.stride[2];
+    prm.k_sg = prm.v_sg = 0;
+    prm.seg_kv = (int)a.k.shape[1];
+  }
+  if (prm.seg_kv <= 0) prm.seg_kv = 1;
   prm.out = a.out.data;
   prm.out_bf16 = a.out.dtype == CP_BF16;
   prm.merge = a.merge ? 1 : 0;
@@ -211,6 +230,8 @@ int launch_attn_ring_f32(const RingArgs& a, cudaStream_t stream) {
   prm.n_row_blocks = (prm.S_q + kRowsPerBlock - 1) / kRowsPerBlock;
   prm.n_chunks = a.n_chunks;
   for (int c = 0; c <= a.n_chunks; ++c) prm.chunk_off[c] = (int)a.chunk_off[c];
+  for (int c = 0; c < a.n_chunks; ++c)
+    prm.chunk_end[c] = (int)(a.chunk_end ? a.chunk_end[c] : a.chunk_off[c + 1]);
   prm.scale = a.scale;
   const long long grid = (long long)prm.n_row_blocks * prm.H * prm.B;
   if (grid <= 0) return CP_OK;

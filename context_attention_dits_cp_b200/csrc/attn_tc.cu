@@ -90,18 +90,21 @@ struct AttnTcParams {
   int n_tiles;                   // key tiles over all chunks
   int n_chunks;
   float scale_log2;              // scale * log2(e)
-  int chunk_off[CP_MAX_CHUNKS + 1];
+  int chunk_off[CP_MAX_CHUNKS + 1];   // chunk c covers key tokens [chunk_off[c], chunk_end[c])
+  int chunk_end[CP_MAX_CHUNKS];
 };
 
 // Walks the key tiles chunk by chunk: [start, start+128) clipped to the
-// chunk end; empty chunks are skipped.
+// chunk end; empty chunks are skipped.  Chunks need not be adjacent: in a
+// padded all-gather buffer the rows between one chunk's end and the next
+// chunk's start are padding, never attended.
 struct TileWalk {
   int c, start, end;
   __device__ __forceinline__ void skip_empty(const AttnTcParams& p) {
-    while (c < p.n_chunks && p.chunk_off[c + 1] <= p.chunk_off[c]) ++c;
+    while (c < p.n_chunks && p.chunk_end[c] <= p.chunk_off[c]) ++c;
     if (c < p.n_chunks) {
       start = p.chunk_off[c];
-      end = p.chunk_off[c + 1];
+      end = p.chunk_end[c];
     }
   }
   __device__ __forceinline__ void init(const AttnTcParams& p) {
@@ -610,12 +613,15 @@ int launch_attn_ring_tc(const RingArgs& a, cudaStream_t stream) {
     prm.seg_q = (int)a.q.shape[2];
     prm.S_q = (int)(a.q.shape[0] * a.q.shape[2]);
     prm.H = (int)a.q.shape[3];
-    prm.seg_kv = (int)a.k.shape[2];
-    prm.S_kv = (int)(a.k.shape[0] * a.k.shape[2]);
   } else {
     prm.B = (int)a.q.shape[0];
     prm.S_q = prm.seg_q = (int)a.q.shape[1];
     prm.H = (int)a.q.shape[2];
+  }
+  if (a.k.ndim == 5) {   // [G, B, L, H, D]: shards, or the slots of a padded all-gather
+    prm.seg_kv = (int)a.k.shape[2];
+    prm.S_kv = (int)(a.k.shape[0] * a.k.shape[2]);
+  } else {
     prm.S_kv = prm.seg_kv = (int)a.k.shape[1];
   }
   if (prm.seg_q <= 0) prm.seg_q = 1;
@@ -625,8 +631,9 @@ int launch_attn_ring_tc(const RingArgs& a, cudaStream_t stream) {
   int n_tiles = 0;
   for (int c = 0; c <= a.n_chunks; ++c) prm.chunk_off[c] = (int)a.chunk_off[c];
   for (int c = 0; c < a.n_chunks; ++c) {
-    const int len = (int)(a.chunk_off[c + 1] - a.chunk_off[c]);
-    n_tiles += (len + kBlockN - 1) / kBlockN;
+    prm.chunk_end[c] = (int)(a.chunk_end ? a.chunk_end[c] : a.chunk_off[c + 1]);
+    const int len = prm.chunk_end[c] - prm.chunk_off[c];
+    if (len > 0) n_tiles += (len + kBlockN - 1) / kBlockN;
   }
   prm.n_tiles = n_tiles;
   prm.scale_log2 = a.scale * 1.4426950408889634f;

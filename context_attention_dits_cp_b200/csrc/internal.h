@@ -34,10 +34,11 @@ inline int dtype_size(int dt) { return dt == CP_BF16 ? 2 : 4; }
 
 // Attention over a chunk list (one chunk = cp_attn_partial).
 struct RingArgs {
-  TensorView q, k, v;      // [B, S, H, D]
+  TensorView q, k, v;      // [B, S, H, D]; k, v may be [G, B, L, H, D] (token s = row s % L of slot s / L)
   TensorView out;          // [B, S_q, H, D] f32 or bf16
   TensorView lse;          // [B, H, S_q] f32; data may be null
-  const int64_t* chunk_off = nullptr;   // host, n_chunks + 1
+  const int64_t* chunk_off = nullptr;   // host, n_chunks + 1: chunk starts (key tokens)
+  const int64_t* chunk_end = nullptr;   // host, n_chunks chunk ends; null: chunk_off[c + 1]
   int n_chunks = 0;
   float scale = 0.f;
   bool merge = false;      // fold into (out, lse) with the fp32 LSE merge

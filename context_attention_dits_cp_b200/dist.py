@@ -1,0 +1,153 @@
+"""Context-parallel attention across ranks (one process per GPU).
+
+The single-GPU calls of this package walk the ring and permute the Ulysses
+layout inside one device.  This module runs the same computation with the
+sequence really sharded over the ranks of a process group, following the
+diffusers context-parallelism guide (§Ring Attention with an all-gather of
+K/V, §Ring Anything for uneven shards, §Ulysses Attention):
+
+* ``ring_attention_allgather`` -- every rank holds its own sequence shard of
+  q, k, v, of any length (Ring Anything).  The shard lengths travel over a
+  CPU group first, so no device synchronisation is needed for metadata.  Each
+  rank pads K/V to the longest shard (padding zeroed), all-gathers them, and
+  attends its queries to every chunk; the padding is trimmed by the chunk
+  walk itself (``cp_ring_attention_gathered`` reads the gathered slots in
+  place).  The local chunk is folded in from local memory while the
+  all-gather is in flight, so the exchange overlaps that compute.
+* ``ulysses_attention_all_to_all`` -- every rank holds S/U tokens of all H
+  heads.  The heads are packed into U groups, exchanged with one all-to-all
+  so that every rank holds all tokens of H/U heads, attended in the shard
+  layout in place, and sent back with the inverse all-to-all.
+
+The kernels are reached through ``ops`` (by default the C-ABI binding of this
+package), so the host-side logic can be exercised on CPU ranks.  Every rank
+issues the same collectives in the same order, also on the error paths:
+a shape mismatch is detected from the exchanged metadata, which every rank
+sees in full, and all ranks raise together.
+"""
+from typing import List, Optional, Sequence
+
+import torch
+import torch.distributed as dist
+
+from . import binding
+
+_DTYPE_CODES = {torch.float32: 0, torch.bfloat16: 1}
+
+
+class ShardMismatch(ValueError):
+    """The ranks' shards disagree on batch, heads, head dim or dtype."""
+
+
+def exchange_shard_meta(q: torch.Tensor, k: torch.Tensor, group=None) -> List[List[int]]:
+    """All ranks' (kv_len, q_len, B, H, D, dtype) rows, gathered over ``group``
+    (a CPU group: the rows are host integers).  Raises ShardMismatch on every
+    rank when B, H, D or the dtype differ, or when q and k of one rank do."""
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q and k must be [B, S, H, D]")
+    code = _DTYPE_CODES.get(q.dtype, -1)
+    bad = int(tuple(k.shape[0:1]) + tuple(k.shape[2:]) != tuple(q.shape[0:1]) + tuple(q.shape[2:])
+              or k.dtype != q.dtype)
+    meta = torch.tensor([k.shape[1], q.shape[1], q.shape[0], q.shape[2], q.shape[3], code, bad],
+                        dtype=torch.int64)
+    world = dist.get_world_size(group)
+    # a CPU group keeps this off the device; over NCCL it costs one sync
+    dev = (torch.device("cuda", torch.cuda.current_device())
+           if dist.get_backend(group) == "nccl" else torch.device("cpu"))
+    meta = meta.to(dev)
+    rows = torch.empty(world * meta.numel(), dtype=torch.int64, device=dev)
+    dist.all_gather_into_tensor(rows, meta, group=group)
+    table = rows.view(world, -1).cpu().tolist()
+    if any(r[6] for r in table):
+        raise ShardMismatch(f"q and k disagree on some rank: {table}")
+    if any(r[2:6] != table[0][2:6] for r in table):
+        raise ShardMismatch(f"ranks disagree on (B, H, D, dtype): {[r[2:6] for r in table]}")
+    return [r[:6] for r in table]
+
+
+def ring_attention_allgather(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, group=None,
+                             cpu_group=None, scale: Optional[float] = None, ops=None):
+    """Attention of this rank's queries to the whole sharded sequence.
+
+    q, k, v: this rank's shard [B, s_r, H, D]; s_r may differ across ranks.
+    group:   the device group (NCCL) that carries K/V; cpu_group: the group
+             that carries the shard lengths (gloo; defaults to ``group``).
+    Returns (out [B, s_q, H, D] fp32, lse [B, H, s_q] fp32) for the local
+    queries against all ranks' keys, chunks merged in rank order.
+    """
+    ops = binding if ops is None else ops
+    rank = dist.get_rank(group)
+    meta = exchange_shard_meta(q, k, cpu_group if cpu_group is not None else group)
+    lengths = [m[0] for m in meta]
+    L = max(lengths)
+    B, s, H, D = k.shape
+    # Ring Anything: pad K/V to the longest shard; padding rows are zeroed
+    # (the gathered-ring call needs them finite), then all-gather [K; V].
+    send = torch.empty((2, B, L, H, D), dtype=k.dtype, device=k.device)
+    send[0, :, :s].copy_(k)
+    send[1, :, :s].copy_(v)
+    if s < L:
+        send[:, :, s:].zero_()
+    recv = torch.empty(len(lengths) * send.numel(), dtype=k.dtype, device=k.device)
+    work = dist.all_gather_into_tensor(recv, send.view(-1), group=group, async_op=True)
+    recv = recv.view(len(lengths), 2, B, L, H, D)
+    # the local chunk needs no exchange: fold it in while K/V travel
+    out, lse = ops.attn_partial(q, k, v, scale=scale)
+    work.wait()
+    ops.ring_attention_gathered(q, recv[:, 0], recv[:, 1], lengths, skip_chunk=rank, scale=scale,
+                                out=out, lse=lse, accumulate=True)
+    return out, lse
+
+
+def _rank_offsets(sizes: Sequence[int]) -> List[int]:
+    off = [0]
+    for n in sizes:
+        off.append(off[-1] + n)
+    return off
+
+
+def ulysses_attention_all_to_all(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, group=None,
+                                 cpu_group=None, scale: Optional[float] = None, ops=None,
+                                 want_lse: bool = False):
+    """Ulysses attention over the ranks of ``group``.
+
+    q, k, v: this rank's S/U tokens of all H heads, [B, S/U, H, D]; every rank
+    holds the same number of tokens and H % U == 0.  Returns this rank's
+    output tokens [B, S/U, H, D] in fp32 (and, with want_lse, the LSE of this
+    rank's head group over the whole sequence, [B, H/U, S]).
+    """
+    ops = binding if ops is None else ops
+    U = dist.get_world_size(group)
+    meta = exchange_shard_meta(q, k, cpu_group if cpu_group is not None else group)
+    if any(m[0] != meta[0][0] or m[1] != meta[0][0] for m in meta):
+        raise ShardMismatch(f"Ulysses needs equal shards on every rank: {meta}")
+    B, Sl, H, D = q.shape
+    if H % U:
+        raise ShardMismatch(f"{H} heads do not split over {U} ranks")
+    Hg = H // U
+    # pack: this rank's tokens of head group g go to rank g.  As an uneven
+    # permutation, the sequence side is one buffer holding all Sl tokens and
+    # the head side is U buffers of Hg heads: [U, B, Sl, Hg, D].
+    seq_off = [0] + [Sl] * U
+    head_off = _rank_offsets([Hg] * U)
+    recvs = []
+    for t in (q, k, v):
+        packed = torch.empty((U, B, Sl, Hg, D), dtype=t.dtype, device=t.device)
+        ops.ulysses_anything_permute(t.reshape(-1), B, H, D, seq_off, head_off,
+                                     binding.SEQ_TO_HEAD, y=packed.view(-1))
+        r = torch.empty_like(packed)
+        dist.all_to_all_single(r, packed, group=group)
+        recvs.append(r)
+    # recv[p] = rank p's tokens of this rank's heads: the shard layout
+    # [U, B, Sl, Hg, D] of the whole sequence, attended in place
+    out_sh = torch.empty((U, B, Sl, Hg, D), dtype=torch.float32, device=q.device)
+    lse = (torch.empty((B, Hg, U * Sl), dtype=torch.float32, device=q.device)
+           if want_lse else None)
+    ops.usp_attention(*recvs, U, 1, scale=scale, out=out_sh, lse=lse, want_lse=want_lse)
+    back = torch.empty_like(out_sh)
+    dist.all_to_all_single(back, out_sh, group=group)
+    # unpack: back[g] holds this rank's tokens of head group g
+    out = torch.empty((B, Sl, H, D), dtype=torch.float32, device=q.device)
+    ops.ulysses_anything_permute(back.view(-1), B, H, D, seq_off, head_off,
+                                 binding.HEAD_TO_SEQ, y=out.view(-1))
+    return (out, lse) if want_lse else out

@@ -75,7 +75,8 @@ enum {
   CP_ERR_ALIGN = -4,     /* base/stride not 16-byte aligned, or inner dim
                             not contiguous                                   */
   CP_ERR_OFFSETS = -5,   /* chunk offsets not monotone, not starting at 0,
-                            not ending at S_kv, or too many chunks           */
+                            not ending at S_kv, or too many chunks; chunk
+                            lengths outside [0, L] or a bad skip_chunk     */
   CP_ERR_DEGREE = -6,    /* Ulysses/ring degree does not divide S or H      */
   CP_ERR_CUDA = -7,      /* a CUDA runtime/driver call failed               */
   CP_ERR_TIMEOUT = -8,   /* a bounded device-side wait gave up              */
@@ -142,6 +143,33 @@ int cp_ring_attention(const cp_tensor* q, const cp_tensor* k,
                       const cp_tensor* v, const int64_t* chunk_offsets,
                       int n_chunks, float scale, cp_tensor* out,
                       cp_tensor* lse, void* stream);
+
+/*
+ * cp_ring_attention_gathered -- the ring over the slots of a padded K/V
+ * all-gather (§Ring Anything: every rank pads its K/V to the longest local
+ * length, the padded shards are all-gathered, and the padding is trimmed
+ * before attention).  Here the trim is part of the chunk walk: chunk c is
+ * rows [0, chunk_lengths[c]) of slot c, read in place, and the padding rows
+ * are never attended.
+ *   q          [B, S_q, H, D]        bf16 or f32
+ *   k_gathered [R, B, L, H, D]       same dtype as q; R = n_chunks slots of
+ *   v_gathered [R, B, L, H, D]       L >= every chunk length (rank order)
+ *   chunk_lengths: HOST array of n_chunks int64 in [0, L].
+ *   skip_chunk: a chunk to leave out (-1: none), typically the caller's own
+ *               chunk when it has already been folded in from local memory.
+ *   accumulate: 0 writes (out, lse) like cp_ring_attention (lse may be
+ *               NULL); 1 folds the result into the fp32 accumulator
+ *               (out f32, lse required) like cp_attn_partial_merge, and is
+ *               a no-op when no chunk remains.
+ * The bf16 path reads whole 128-row tiles, so the padding rows of v inside
+ * a chunk's last tile are multiplied by exact zeros: they must be finite
+ * (zero them when padding).  Padding of k may hold anything.
+ */
+int cp_ring_attention_gathered(const cp_tensor* q, const cp_tensor* k_gathered,
+                               const cp_tensor* v_gathered,
+                               const int64_t* chunk_lengths, int n_chunks,
+                               int skip_chunk, float scale, int accumulate,
+                               cp_tensor* out, cp_tensor* lse, void* stream);
 
 /*
  * cp_ulysses_permute -- the Ulysses all-to-all as an on-GPU layout

@@ -107,6 +107,29 @@ def test_self_overlapping_outputs_are_rejected():
     assert L.cp_ulysses_permute(r(x), r(y), 2, 0, None) == -10
 
 
+def test_gathered_ring_errors():
+    q, k, v, out, lse = _ok_args()
+    L = bd.lib()
+    r = ctypes.byref
+    kg = _t([4, 1, 96, 2, 128], bd.CP_BF16, FAKE + (1 << 24))
+    vg = _t([4, 1, 96, 2, 128], bd.CP_BF16, FAKE + (2 << 24))
+    lens = (ctypes.c_int64 * 4)(96, 0, 50, 7)
+    call = lambda lens, n, skip, acc, o=out, l=lse: L.cp_ring_attention_gathered(
+        r(q), r(kg), r(vg), lens, n, skip, 0.0, acc, r(o), r(l) if l is not None else None, None)
+    assert call(lens, 3, -1, 0) == -5                                   # n_chunks != slots
+    assert call(lens, 4, 4, 0) == -5                                    # skip out of range
+    assert call(lens, 4, -2, 0) == -5
+    assert call((ctypes.c_int64 * 4)(97, 0, 50, 7), 4, -1, 0) == -5    # longer than a slot
+    assert call((ctypes.c_int64 * 4)(-1, 0, 50, 7), 4, -1, 0) == -5
+    assert call(None, 4, -1, 0) == -1
+    bf_out = _t([1, 256, 2, 128], bd.CP_BF16, FAKE + (3 << 24))
+    assert call(lens, 4, -1, 1, o=bf_out) == -2                         # accumulator is f32
+    assert call(lens, 4, -1, 1, l=None) == -1                           # and needs its lse
+    k4 = _t([1, 300, 2, 128], bd.CP_BF16, FAKE + (1 << 24))
+    assert L.cp_ring_attention_gathered(r(q), r(k4), r(vg), lens, 4, -1, 0.0, 0, r(out),
+                                        r(lse), None) == -3             # slots are 5-D
+
+
 def test_partial_merge_errors():
     q, k, v, out, lse = _ok_args()
     L = bd.lib()

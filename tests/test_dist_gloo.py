@@ -1,0 +1,158 @@
+"""Multi-rank context parallelism (context_attention_dits_cp_b200.dist) as
+world-size-2 gloo ranks on the CPU.
+
+The host logic runs unchanged: the shard-length exchange, the Ring Anything
+padding and all-gather, the skip of the local chunk, the Ulysses packing,
+all-to-alls and unpacking.  The kernel calls go to a stand-in built from the
+oracle (this file), since the CUDA kernels need a GPU; the GPU side of the
+same calls is covered by the parity tests.  Results are compared with
+one-shot attention over the whole sequence."""
+import os
+import socket
+import sys
+import traceback
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+class OracleOps:
+    """The kernel entry points dist.py calls, computed by the fp64 oracle on
+    CPU tensors (results stored as fp32, like the kernels' outputs)."""
+
+    def __init__(self, oracle):
+        self.o = oracle
+
+    @staticmethod
+    def _np(t):
+        return t.detach().double().numpy()
+
+    def attn_partial(self, q, k, v, scale=None):
+        out, lse = self.o.attention_partial(self._np(q), self._np(k), self._np(v), scale)
+        return torch.from_numpy(out).float(), torch.from_numpy(lse).float()
+
+    def ring_attention_gathered(self, q, kg, vg, lengths, skip_chunk=-1, scale=None, out=None,
+                                lse=None, accumulate=False):
+        assert accumulate and out is not None and lse is not None
+        acc, lacc = self._np(out), self._np(lse)
+        for c, n in enumerate(lengths):
+            if c == skip_chunk or n == 0:
+                continue
+            oc, lc = self.o.attention_partial(self._np(q), self._np(kg[c, :, :n]),
+                                              self._np(vg[c, :, :n]), scale)
+            acc, lacc = self.o.lse_merge(acc, lacc, oc, lc)
+        out.copy_(torch.from_numpy(acc))
+        lse.copy_(torch.from_numpy(lacc))
+        return out, lse
+
+    def ulysses_anything_permute(self, x, B, H, D, seq_off, head_off, direction, y=None):
+        r = self.o.ulysses_anything_permute(x.numpy(), B, H, D, seq_off, head_off, direction)
+        y.copy_(torch.from_numpy(np.ascontiguousarray(r)).reshape(y.shape))
+        return y
+
+    def usp_attention(self, qs, ks, vs, R, U, scale=None, out=None, lse=None, want_lse=True):
+        o, l = self.o.usp_attention(self._np(qs), self._np(ks), self._np(vs), R, U, scale)
+        out.copy_(torch.from_numpy(o))
+        if lse is not None:
+            lse.copy_(torch.from_numpy(l))
+        return out, lse
+
+
+def _worker(rank, world, port, case, q):
+    try:
+        sys.path.insert(0, ROOT)
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+        import datetime
+        dist.init_process_group("gloo", rank=rank, world_size=world,
+                                timeout=datetime.timedelta(seconds=60))
+        import oracle
+        from context_attention_dits_cp_b200 import dist as cpd
+        from context_attention_dits_cp_b200 import workloads as wl
+        ops = OracleOps(oracle)
+        if case == "ring":
+            # Ring Anything: uneven shards (and an uneven query split)
+            kv_len, q_len, H, D = [37, 29], [20, 33], 3, 16
+            qa, ka, va = wl.make_qkv(2, H, sum(q_len), D, torch.float32, 71, S_kv=sum(kv_len))
+            qo, ko = sum(q_len[:rank]), sum(kv_len[:rank])
+            ql = qa[:, qo:qo + q_len[rank]]
+            kl = ka[:, ko:ko + kv_len[rank]].contiguous()
+            vl = va[:, ko:ko + kv_len[rank]].contiguous()
+            out, lse = cpd.ring_attention_allgather(ql, kl, vl, ops=ops)
+            ro, rl = oracle.attention(qa.double().numpy(), ka.double().numpy(),
+                                      va.double().numpy())
+            eo = float(np.abs(out.numpy() - ro[:, qo:qo + q_len[rank]]).max())
+            el = float(np.abs(lse.numpy() - rl[:, :, qo:qo + q_len[rank]]).max())
+            q.put((rank, "ok", eo, el))
+        elif case == "ulysses":
+            B, S, H, D = 2, 10, 4, 8
+            qa, ka, va = wl.make_qkv(B, H, S, D, torch.float32, 72)
+            Sl = S // world
+            sl = slice(rank * Sl, (rank + 1) * Sl)
+            out, lse = cpd.ulysses_attention_all_to_all(qa[:, sl].contiguous(),
+                                                        ka[:, sl].contiguous(),
+                                                        va[:, sl].contiguous(), ops=ops,
+                                                        want_lse=True)
+            ro, rl = oracle.attention(qa.double().numpy(), ka.double().numpy(),
+                                      va.double().numpy())
+            Hg = H // world
+            eo = float(np.abs(out.numpy() - ro[:, sl]).max())
+            el = float(np.abs(lse.numpy() - rl[:, rank * Hg:(rank + 1) * Hg]).max())
+            q.put((rank, "ok", eo, el))
+        elif case == "mismatch":
+            # rank 1 holds a different number of heads: every rank must raise
+            H = 3 if rank == 0 else 4
+            qa, ka, va = wl.make_qkv(1, H, 8, 16, torch.float32, 73)
+            try:
+                cpd.ring_attention_allgather(qa, ka, va, ops=ops)
+                q.put((rank, "no error", 0.0, 0.0))
+            except cpd.ShardMismatch:
+                q.put((rank, "raised", 0.0, 0.0))
+        dist.destroy_process_group()
+    except Exception:
+        q.put((rank, "crash: " + traceback.format_exc(), 0.0, 0.0))
+        raise
+
+
+def _run(case, world=2):
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, case, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+    res = sorted(q.get(timeout=5) for _ in range(world))
+    assert all(p.exitcode == 0 for p in procs), res
+    return res
+
+
+def test_ring_allgather_uneven_shards_equals_oneshot():
+    for rank, status, eo, el in _run("ring"):
+        assert status == "ok", status
+        assert eo <= 1e-5 and el <= 1e-5, (rank, eo, el)
+
+
+def test_ulysses_all_to_all_equals_oneshot():
+    for rank, status, eo, el in _run("ulysses"):
+        assert status == "ok", status
+        assert eo <= 1e-5 and el <= 1e-5, (rank, eo, el)
+
+
+def test_shape_mismatch_raises_on_every_rank():
+    res = _run("mismatch")
+    assert [r[1] for r in res] == ["raised", "raised"], res

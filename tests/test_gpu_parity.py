@@ -271,6 +271,61 @@ def test_partial_merge_into_strided_views(cuda_ok, dtype):
     assert bool((lbig[:, :, :10] == 3.0).all()) and bool((lbig[:, :, 10 + Sq:] == 3.0).all())
 
 
+def _padded_gather(t, lengths, L, pad):
+    """[R, B, L, H, D] slots of a padded all-gather of the chunks of t
+    (rank order), padding rows set to `pad`."""
+    B, _, H, D = t.shape
+    g = torch.full((len(lengths), B, L, H, D), pad, dtype=t.dtype)
+    o = 0
+    for c, n in enumerate(lengths):
+        g[c, :, :n] = t[:, o:o + n]
+        o += n
+    return g
+
+
+@pytest.mark.parametrize("dtype,D,B", [(torch.bfloat16, 128, 1), (torch.bfloat16, 64, 2),
+                                       (torch.float32, 128, 2)])
+def test_gathered_ring_trims_padding_in_place(cuda_ok, dtype, D, B):
+    """Ring Anything over a padded all-gather: chunk c is the first
+    lengths[c] rows of slot c; the padding (NaN in K, 1e30 in V) never
+    contributes.  Whole walk, and own chunk first then the rest merged in."""
+    lengths, L, H, Sq = [300, 0, 257, 128], 320, 3, 290
+    Skv = sum(lengths)
+    q, k, v = wl.make_qkv(B, H, Sq, D, dtype, 61, "kscale", S_kv=Skv)
+    kg = _padded_gather(k, lengths, L, float("nan")).cuda()
+    vg = _padded_gather(v, lengths, L, 1e30).cuda()
+    dq = q.cuda()
+    ro, rl = oracle.attention(_np(q), _np(k), _np(v))
+    out, lse = cp.ring_attention_gathered(dq, kg, vg, lengths)
+    torch.cuda.synchronize()
+    _check(out, lse, ro, rl, dtype)
+    # rank 2 folds in its own chunk first, then the others from the gather
+    r = 2
+    o0 = sum(lengths[:r])
+    acc, lacc = cp.attn_partial(dq, k[:, o0:o0 + lengths[r]].cuda(), v[:, o0:o0 + lengths[r]].cuda())
+    cp.ring_attention_gathered(dq, kg, vg, lengths, skip_chunk=r, out=acc, lse=lacc,
+                               accumulate=True)
+    torch.cuda.synchronize()
+    _check(acc, lacc, ro, rl, dtype)
+
+
+def test_gathered_ring_empty_cases(cuda_ok):
+    """No chunk left: accumulate leaves the accumulator alone, otherwise the
+    result is attention to no keys (0, -inf)."""
+    q, k, v = wl.make_qkv(1, 2, 130, 128, torch.bfloat16, 62, S_kv=40)
+    kg = _padded_gather(k, [40, 0], 64, 0.0).cuda()
+    vg = _padded_gather(v, [40, 0], 64, 0.0).cuda()
+    acc = torch.randn(1, 130, 2, 128, device="cuda")
+    lacc = torch.randn(1, 2, 130, device="cuda")
+    a0, l0 = acc.clone(), lacc.clone()
+    cp.ring_attention_gathered(q.cuda(), kg, vg, [40, 0], skip_chunk=0, out=acc, lse=lacc,
+                               accumulate=True)
+    out, lse = cp.ring_attention_gathered(q.cuda(), kg, vg, [40, 0], skip_chunk=0)
+    torch.cuda.synchronize()
+    assert torch.equal(acc, a0) and torch.equal(lacc, l0)
+    assert bool((out == 0).all()) and bool(torch.isneginf(lse).all())
+
+
 def test_constant_v_and_zero_q_closed_forms(cuda_ok):
     g = torch.Generator().manual_seed(18)
     S = 400
