@@ -371,6 +371,30 @@ def run_cuda(args):
         "launches": w.ring_degree, "ms": float(np.mean(t_r)), "TFLOP/s": tf,
         "frac_of_bf16_peak": tf / tc_peak,
         "vs_single_launch": float(kernel_ms / np.mean(t_r))}
+    # Ring Anything over ranks, as rank 0 sees it after the padded all-gather:
+    # FLUX keys in 4 uneven shards (1172, 1172, 1172, 1092) padded to 1172;
+    # own chunk first from local memory, then the other three slots
+    g_len = [1172, 1172, 1172, 1092]
+    g_pad = max(g_len)
+    kg = torch.zeros((4, w.B, g_pad, w.H, w.D), dtype=dk.dtype, device=dev)
+    vg = torch.zeros_like(kg)
+    o = 0
+    for c, n in enumerate(g_len):
+        kg[c, :, :n] = dk[:, o:o + n]
+        vg[c, :, :n] = dv[:, o:o + n]
+        o += n
+
+    def gathered_ring():
+        cp.attn_partial(dq, kg[0, :, :g_len[0]], vg[0, :, :g_len[0]], out=out, lse=lse)
+        cp.ring_attention_gathered(dq, kg, vg, g_len, skip_chunk=0, out=out, lse=lse,
+                                   accumulate=True)
+
+    t_g = _time_loop(gathered_ring, n_merge, 3, flush, stream)
+    tf = flops / (np.mean(t_g) * 1e-3) / 1e12
+    components["ring_gathered_uneven_own_chunk_first"] = {
+        "lengths": g_len, "launches": 2, "ms": float(np.mean(t_g)), "TFLOP/s": tf,
+        "frac_of_bf16_peak": tf / tc_peak}
+    del kg, vg
     # unified R=2 x U=2 grid (B=2, S=8192, H=24, D=128) from sequence shards
     uq, uk, uv = wl.make_workload_inputs(u)
     ush = [wl.sequence_shards(t, 4).to(dev) for t in (uq, uk, uv)]
