@@ -75,7 +75,8 @@ def _worker(rank, world, port, case, q):
         os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
         import datetime
         dist.init_process_group("gloo", rank=rank, world_size=world,
-                                timeout=datetime.timedelta(seconds=60))
+                                timeout=datetime.timedelta(seconds=5 if case == "rank_leaves"
+                                                           else 60))
         import oracle
         from context_attention_dits_cp_b200 import dist as cpd
         from context_attention_dits_cp_b200 import workloads as wl
@@ -109,6 +110,26 @@ def _worker(rank, world, port, case, q):
             eo = float(np.abs(out.numpy() - ro[:, sl]).max())
             el = float(np.abs(lse.numpy() - rl[:, rank * Hg:(rank + 1) * Hg]).max())
             q.put((rank, "ok", eo, el))
+        elif case == "rank_leaves":
+            # rank 1 leaves between steps without joining the exchange: rank 0's
+            # metadata all-gather must end with an error within the group's
+            # timeout instead of waiting for good
+            if rank == 1:
+                q.put((rank, "left", 0.0, 0.0))
+                q.close()
+                q.join_thread()
+                os._exit(0)
+            import time
+            qa, ka, va = wl.make_qkv(1, 2, 8, 16, torch.float32, 74)
+            t0 = time.monotonic()
+            try:
+                cpd.ring_attention_allgather(qa, ka, va, ops=ops)
+                q.put((rank, "no error", 0.0, 0.0))
+            except RuntimeError:
+                q.put((rank, "raised", time.monotonic() - t0, 0.0))
+            q.close()
+            q.join_thread()
+            os._exit(0)
         elif case == "mismatch":
             # rank 1 holds a different number of heads: every rank must raise
             H = 3 if rank == 0 else 4
@@ -124,7 +145,7 @@ def _worker(rank, world, port, case, q):
         raise
 
 
-def _run(case, world=2):
+def _run(case, world=2, allow_exit=False):
     port = _free_port()
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
@@ -139,6 +160,13 @@ def _run(case, world=2):
     res = sorted(q.get(timeout=5) for _ in range(world))
     assert all(p.exitcode == 0 for p in procs), res
     return res
+
+
+def test_a_rank_that_leaves_ends_the_others_collective_with_an_error():
+    res = _run("rank_leaves")
+    assert res[1][1] == "left"
+    assert res[0][1] == "raised", res
+    assert res[0][2] < 60.0          # bounded by the group's 5 s timeout, not a hang
 
 
 def test_ring_allgather_uneven_shards_equals_oneshot():
