@@ -14,10 +14,13 @@ K/V, §Ring Anything for uneven shards, §Ulysses Attention):
   walk itself (``cp_ring_attention_gathered`` reads the gathered slots in
   place).  The local chunk is folded in from local memory while the
   all-gather is in flight, so the exchange overlaps that compute.
-* ``ulysses_attention_all_to_all`` -- every rank holds S/U tokens of all H
+* ``ulysses_attention_all_to_all`` -- every rank holds its tokens of all H
   heads.  The heads are packed into U groups, exchanged with one all-to-all
-  so that every rank holds all tokens of H/U heads, attended in the shard
-  layout in place, and sent back with the inverse all-to-all.
+  so that every rank holds all tokens of its head group, attended, and sent
+  back with the inverse all-to-all.  Equal shards with H % U == 0 are the
+  guide's Ulysses (attended in the shard layout in place); anything else is
+  Ulysses Anything (§Ulysses Anything): uneven shards, heads split as
+  ceil(H/U) per rank, exchanged with uneven all-to-all splits.
 
 The kernels are reached through ``ops`` (by default the C-ABI binding of this
 package), so the host-side logic can be exercised on CPU ranks.  Every rank
@@ -111,43 +114,63 @@ def ulysses_attention_all_to_all(q: torch.Tensor, k: torch.Tensor, v: torch.Tens
                                  want_lse: bool = False):
     """Ulysses attention over the ranks of ``group``.
 
-    q, k, v: this rank's S/U tokens of all H heads, [B, S/U, H, D]; every rank
-    holds the same number of tokens and H % U == 0.  Returns this rank's
-    output tokens [B, S/U, H, D] in fp32 (and, with want_lse, the LSE of this
-    rank's head group over the whole sequence, [B, H/U, S]).
+    q, k, v: this rank's tokens of all H heads, [B, s_r, H, D].  With equal
+    shards and H % U == 0 this is the guide's Ulysses; otherwise Ulysses
+    Anything: the shards may differ in length and the heads split as
+    ceil(H/U) per rank, the last ranks holding fewer (possibly none).
+    Returns this rank's output tokens [B, s_r, H, D] in fp32 (and, with
+    want_lse, the LSE of this rank's head group over the whole sequence,
+    [B, h_r, S]).
     """
     ops = binding if ops is None else ops
     U = dist.get_world_size(group)
+    me = dist.get_rank(group)
     meta = exchange_shard_meta(q, k, cpu_group if cpu_group is not None else group)
-    if any(m[0] != meta[0][0] or m[1] != meta[0][0] for m in meta):
-        raise ShardMismatch(f"Ulysses needs equal shards on every rank: {meta}")
-    B, Sl, H, D = q.shape
-    if H % U:
-        raise ShardMismatch(f"{H} heads do not split over {U} ranks")
-    Hg = H // U
+    if any(m[0] != m[1] for m in meta):
+        raise ShardMismatch(f"Ulysses needs q and k/v of one length on every rank: {meta}")
+    B, s, H, D = q.shape
+    lens = [m[0] for m in meta]
+    seq_off = _rank_offsets(lens)
+    head_off = binding.ring_chunk_offsets(H, U)
+    heads = [head_off[g + 1] - head_off[g] for g in range(U)]
     # pack: this rank's tokens of head group g go to rank g.  As an uneven
-    # permutation, the sequence side is one buffer holding all Sl tokens and
-    # the head side is U buffers of Hg heads: [U, B, Sl, Hg, D].
-    seq_off = [0] + [Sl] * U
-    head_off = _rank_offsets([Hg] * U)
+    # permutation, the sequence side is one buffer holding all s tokens and
+    # the head side is U buffers of heads[g] heads.
+    one = [0] + [s] * U
+    send_n = [B * s * heads[g] * D for g in range(U)]
+    recv_n = [B * lens[p] * heads[me] * D for p in range(U)]
+    even = all(n == lens[0] for n in lens) and H % U == 0
     recvs = []
     for t in (q, k, v):
-        packed = torch.empty((U, B, Sl, Hg, D), dtype=t.dtype, device=t.device)
-        ops.ulysses_anything_permute(t.reshape(-1), B, H, D, seq_off, head_off,
-                                     binding.SEQ_TO_HEAD, y=packed.view(-1))
-        r = torch.empty_like(packed)
-        dist.all_to_all_single(r, packed, group=group)
+        packed = torch.empty(B * s * H * D, dtype=t.dtype, device=t.device)
+        ops.ulysses_anything_permute(t.reshape(-1), B, H, D, one, head_off, binding.SEQ_TO_HEAD,
+                                     y=packed)
+        r = torch.empty(sum(recv_n), dtype=t.dtype, device=t.device)
+        dist.all_to_all_single(r, packed, output_split_sizes=recv_n, input_split_sizes=send_n,
+                               group=group)
         recvs.append(r)
-    # recv[p] = rank p's tokens of this rank's heads: the shard layout
-    # [U, B, Sl, Hg, D] of the whole sequence, attended in place
-    out_sh = torch.empty((U, B, Sl, Hg, D), dtype=torch.float32, device=q.device)
-    lse = (torch.empty((B, Hg, U * Sl), dtype=torch.float32, device=q.device)
-           if want_lse else None)
-    ops.usp_attention(*recvs, U, 1, scale=scale, out=out_sh, lse=lse, want_lse=want_lse)
-    back = torch.empty_like(out_sh)
-    dist.all_to_all_single(back, out_sh, group=group)
-    # unpack: back[g] holds this rank's tokens of head group g
-    out = torch.empty((B, Sl, H, D), dtype=torch.float32, device=q.device)
-    ops.ulysses_anything_permute(back.view(-1), B, H, D, seq_off, head_off,
-                                 binding.HEAD_TO_SEQ, y=out.view(-1))
+    # recv = rank p's tokens of this rank's heads, p in order: the whole
+    # sequence of heads[me] heads, held as U uneven rank buffers
+    Hm = heads[me]
+    if even:
+        # equal shards: the shard layout [U, B, s, Hm, D], attended in place
+        shards = [r.view(U, B, s, Hm, D) for r in recvs]
+        out_sh = torch.empty((U, B, s, Hm, D), dtype=torch.float32, device=q.device)
+        lse = (torch.empty((B, Hm, U * s), dtype=torch.float32, device=q.device)
+               if want_lse else None)
+        ops.usp_attention(*shards, U, 1, scale=scale, out=out_sh, lse=lse, want_lse=want_lse)
+        o_flat = out_sh.view(-1)
+    else:
+        o_flat = torch.empty(sum(recv_n), dtype=torch.float32, device=q.device)
+        lse = (torch.empty((B, Hm, seq_off[-1]), dtype=torch.float32, device=q.device)
+               if want_lse else None)
+        ops.ulysses_anything_attention(*recvs, B, Hm, D, seq_off, [0] + [Hm] * U, scale=scale,
+                                       out=o_flat, lse=lse, want_lse=want_lse)
+    back = torch.empty(B * s * H * D, dtype=torch.float32, device=q.device)
+    dist.all_to_all_single(back, o_flat, output_split_sizes=send_n, input_split_sizes=recv_n,
+                           group=group)
+    # unpack: back holds this rank's tokens of head group g, g in order
+    out = torch.empty((B, s, H, D), dtype=torch.float32, device=q.device)
+    ops.ulysses_anything_permute(back, B, H, D, one, head_off, binding.HEAD_TO_SEQ,
+                                 y=out.view(-1))
     return (out, lse) if want_lse else out

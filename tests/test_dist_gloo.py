@@ -61,6 +61,15 @@ class OracleOps:
         y.copy_(torch.from_numpy(np.ascontiguousarray(r)).reshape(y.shape))
         return y
 
+    def ulysses_anything_attention(self, q, k, v, B, H, D, seq_off, head_off, scale=None,
+                                   out=None, lse=None, want_lse=True):
+        o, l = self.o.ulysses_anything_attention(self._np(q), self._np(k), self._np(v), B, H, D,
+                                                 seq_off, head_off, scale)
+        out.copy_(torch.from_numpy(o))
+        if lse is not None:
+            lse.copy_(torch.from_numpy(l))
+        return out, lse
+
     def usp_attention(self, qs, ks, vs, R, U, scale=None, out=None, lse=None, want_lse=True):
         o, l = self.o.usp_attention(self._np(qs), self._np(ks), self._np(vs), R, U, scale)
         out.copy_(torch.from_numpy(o))
@@ -109,6 +118,24 @@ def _worker(rank, world, port, case, q):
             Hg = H // world
             eo = float(np.abs(out.numpy() - ro[:, sl]).max())
             el = float(np.abs(lse.numpy() - rl[:, rank * Hg:(rank + 1) * Hg]).max())
+            q.put((rank, "ok", eo, el))
+        elif case == "ulysses_uneven":
+            # Ulysses Anything over 3 ranks: 5, 4 and 3 tokens; 4 heads split
+            # 2, 2, 0 (ceil rule), so the last rank attends no heads at all
+            B, H, D, lens = 2, 4, 8, [5, 4, 3]
+            qa, ka, va = wl.make_qkv(B, H, sum(lens), D, torch.float32, 75)
+            o0 = sum(lens[:rank])
+            sl = slice(o0, o0 + lens[rank])
+            out, lse = cpd.ulysses_attention_all_to_all(qa[:, sl].contiguous(),
+                                                        ka[:, sl].contiguous(),
+                                                        va[:, sl].contiguous(), ops=ops,
+                                                        want_lse=True)
+            ro, rl = oracle.attention(qa.double().numpy(), ka.double().numpy(),
+                                      va.double().numpy())
+            h0, h1 = [0, 2, 4, 4][rank], [0, 2, 4, 4][rank + 1]
+            eo = float(np.abs(out.numpy() - ro[:, sl]).max())
+            el = float(np.abs(lse.numpy() - rl[:, h0:h1]).max()) if h1 > h0 else 0.0
+            assert lse.shape == (B, h1 - h0, sum(lens))
             q.put((rank, "ok", eo, el))
         elif case == "rank_leaves":
             # rank 1 leaves between steps without joining the exchange: rank 0's
@@ -177,6 +204,12 @@ def test_ring_allgather_uneven_shards_equals_oneshot():
 
 def test_ulysses_all_to_all_equals_oneshot():
     for rank, status, eo, el in _run("ulysses"):
+        assert status == "ok", status
+        assert eo <= 1e-5 and el <= 1e-5, (rank, eo, el)
+
+
+def test_ulysses_anything_uneven_shards_and_heads_over_three_ranks():
+    for rank, status, eo, el in _run("ulysses_uneven", world=3):
         assert status == "ok", status
         assert eo <= 1e-5 and el <= 1e-5, (rank, eo, el)
 
