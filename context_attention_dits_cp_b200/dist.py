@@ -109,6 +109,53 @@ def _rank_offsets(sizes: Sequence[int]) -> List[int]:
     return off
 
 
+class _HeadExchange:
+    """One rank's side of the Ulysses all-to-all and its inverse.
+
+    scatter(): this rank's tokens of all H heads -> the whole group
+    sequence of this rank's head group, held as U rank buffers
+    [B, s_p, h_me, D] in rank order (flat).  gather(): the inverse, for an
+    fp32 result in that layout.  Heads split ceil(H/U) per rank; shards may
+    differ in length (Ulysses Anything)."""
+
+    def __init__(self, ops, group, meta, B, H, D):
+        self.ops, self.group = ops, group
+        U, me = dist.get_world_size(group), dist.get_rank(group)
+        self.U, self.B, self.H, self.D = U, B, H, D
+        self.lens = [m[0] for m in meta]
+        self.seq_off = _rank_offsets(self.lens)
+        self.head_off = binding.ring_chunk_offsets(H, U)
+        heads = [self.head_off[g + 1] - self.head_off[g] for g in range(U)]
+        self.h_me = heads[me]
+        s = self.lens[me]
+        self.s = s
+        # pack: the sequence side is one buffer holding all s local tokens,
+        # the head side is U buffers of heads[g] heads
+        self.one = [0] + [s] * U
+        self.send_n = [B * s * heads[g] * D for g in range(U)]
+        self.recv_n = [B * self.lens[p] * self.h_me * D for p in range(U)]
+
+    def scatter(self, t):
+        packed = torch.empty(self.B * self.s * self.H * self.D, dtype=t.dtype, device=t.device)
+        self.ops.ulysses_anything_permute(t.reshape(-1), self.B, self.H, self.D, self.one,
+                                          self.head_off, binding.SEQ_TO_HEAD, y=packed)
+        r = torch.empty(sum(self.recv_n), dtype=t.dtype, device=t.device)
+        dist.all_to_all_single(r, packed, output_split_sizes=self.recv_n,
+                               input_split_sizes=self.send_n, group=self.group)
+        return r
+
+    def gather(self, o_flat):
+        back = torch.empty(self.B * self.s * self.H * self.D, dtype=torch.float32,
+                           device=o_flat.device)
+        dist.all_to_all_single(back, o_flat, output_split_sizes=self.send_n,
+                               input_split_sizes=self.recv_n, group=self.group)
+        out = torch.empty((self.B, self.s, self.H, self.D), dtype=torch.float32,
+                          device=o_flat.device)
+        self.ops.ulysses_anything_permute(back, self.B, self.H, self.D, self.one, self.head_off,
+                                          binding.HEAD_TO_SEQ, y=out.view(-1))
+        return out
+
+
 def ulysses_attention_all_to_all(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, group=None,
                                  cpu_group=None, scale: Optional[float] = None, ops=None,
                                  want_lse: bool = False):
@@ -124,35 +171,14 @@ def ulysses_attention_all_to_all(q: torch.Tensor, k: torch.Tensor, v: torch.Tens
     """
     ops = binding if ops is None else ops
     U = dist.get_world_size(group)
-    me = dist.get_rank(group)
     meta = exchange_shard_meta(q, k, cpu_group if cpu_group is not None else group)
     if any(m[0] != m[1] for m in meta):
         raise ShardMismatch(f"Ulysses needs q and k/v of one length on every rank: {meta}")
     B, s, H, D = q.shape
-    lens = [m[0] for m in meta]
-    seq_off = _rank_offsets(lens)
-    head_off = binding.ring_chunk_offsets(H, U)
-    heads = [head_off[g + 1] - head_off[g] for g in range(U)]
-    # pack: this rank's tokens of head group g go to rank g.  As an uneven
-    # permutation, the sequence side is one buffer holding all s tokens and
-    # the head side is U buffers of heads[g] heads.
-    one = [0] + [s] * U
-    send_n = [B * s * heads[g] * D for g in range(U)]
-    recv_n = [B * lens[p] * heads[me] * D for p in range(U)]
-    even = all(n == lens[0] for n in lens) and H % U == 0
-    recvs = []
-    for t in (q, k, v):
-        packed = torch.empty(B * s * H * D, dtype=t.dtype, device=t.device)
-        ops.ulysses_anything_permute(t.reshape(-1), B, H, D, one, head_off, binding.SEQ_TO_HEAD,
-                                     y=packed)
-        r = torch.empty(sum(recv_n), dtype=t.dtype, device=t.device)
-        dist.all_to_all_single(r, packed, output_split_sizes=recv_n, input_split_sizes=send_n,
-                               group=group)
-        recvs.append(r)
-    # recv = rank p's tokens of this rank's heads, p in order: the whole
-    # sequence of heads[me] heads, held as U uneven rank buffers
-    Hm = heads[me]
-    if even:
+    x = _HeadExchange(ops, group, meta, B, H, D)
+    recvs = [x.scatter(t) for t in (q, k, v)]
+    Hm = x.h_me
+    if all(n == x.lens[0] for n in x.lens) and H % U == 0:
         # equal shards: the shard layout [U, B, s, Hm, D], attended in place
         shards = [r.view(U, B, s, Hm, D) for r in recvs]
         out_sh = torch.empty((U, B, s, Hm, D), dtype=torch.float32, device=q.device)
@@ -161,16 +187,57 @@ def ulysses_attention_all_to_all(q: torch.Tensor, k: torch.Tensor, v: torch.Tens
         ops.usp_attention(*shards, U, 1, scale=scale, out=out_sh, lse=lse, want_lse=want_lse)
         o_flat = out_sh.view(-1)
     else:
-        o_flat = torch.empty(sum(recv_n), dtype=torch.float32, device=q.device)
-        lse = (torch.empty((B, Hm, seq_off[-1]), dtype=torch.float32, device=q.device)
+        o_flat = torch.empty(sum(x.recv_n), dtype=torch.float32, device=q.device)
+        lse = (torch.empty((B, Hm, x.seq_off[-1]), dtype=torch.float32, device=q.device)
                if want_lse else None)
-        ops.ulysses_anything_attention(*recvs, B, Hm, D, seq_off, [0] + [Hm] * U, scale=scale,
+        ops.ulysses_anything_attention(*recvs, B, Hm, D, x.seq_off, [0] + [Hm] * U, scale=scale,
                                        out=o_flat, lse=lse, want_lse=want_lse)
-    back = torch.empty(B * s * H * D, dtype=torch.float32, device=q.device)
-    dist.all_to_all_single(back, o_flat, output_split_sizes=send_n, input_split_sizes=recv_n,
-                           group=group)
-    # unpack: back holds this rank's tokens of head group g, g in order
-    out = torch.empty((B, s, H, D), dtype=torch.float32, device=q.device)
-    ops.ulysses_anything_permute(back, B, H, D, one, head_off, binding.HEAD_TO_SEQ,
-                                 y=out.view(-1))
+    out = x.gather(o_flat)
     return (out, lse) if want_lse else out
+
+
+def usp_attention_2d(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ring_group,
+                     ulysses_group, ring_cpu_group=None, ulysses_cpu_group=None,
+                     scale: Optional[float] = None, ops=None):
+    """The unified composition on a 2-D mesh of R x U ranks (ring outer,
+    Ulysses inner: rank g = r * U + u holds sequence shard g).
+
+    1. Ulysses all-to-all inside the Ulysses group: this rank then holds the
+       whole group sequence block for its head group;
+    2. the ring over the ring group: padded all-gather of those blocks,
+       local block first, the rest merged in (ring_attention_allgather);
+    3. the inverse all-to-all.
+    q, k, v: this rank's shard [B, s_g, H, D].  Returns this rank's output
+    tokens [B, s_g, H, D] in fp32.
+    """
+    ops = binding if ops is None else ops
+    U = dist.get_world_size(ulysses_group)
+    meta = exchange_shard_meta(q, k, ulysses_cpu_group if ulysses_cpu_group is not None
+                               else ulysses_group)
+    if any(m[0] != m[1] for m in meta):
+        raise ShardMismatch(f"the unified layout needs q and k/v of one length: {meta}")
+    B, s, H, D = q.shape
+    x = _HeadExchange(ops, ulysses_group, meta, B, H, D)
+    Hm = x.h_me
+    # the Ulysses group's block as one [B, S_u, Hm, D] sequence: the rank
+    # buffers are concatenated along the sequence (free when B == 1)
+    S_u = x.seq_off[-1]
+    blk_heads = [0] + [Hm] * U
+
+    def as_block(r):
+        if B == 1:
+            return r.view(1, S_u, Hm, D)
+        b = torch.empty(B * S_u * Hm * D, dtype=r.dtype, device=r.device)
+        ops.ulysses_anything_permute(r, B, Hm, D, x.seq_off, blk_heads, binding.SEQ_TO_HEAD, y=b)
+        return b.view(B, S_u, Hm, D)
+
+    qb, kb, vb = (as_block(x.scatter(t)) for t in (q, k, v))
+    out_b, _ = ring_attention_allgather(qb, kb, vb, group=ring_group, cpu_group=ring_cpu_group,
+                                        scale=scale, ops=ops)
+    if B == 1:
+        o_flat = out_b.reshape(-1)
+    else:
+        o_flat = torch.empty(B * S_u * Hm * D, dtype=torch.float32, device=q.device)
+        ops.ulysses_anything_permute(out_b.reshape(-1), B, Hm, D, x.seq_off, blk_heads,
+                                     binding.HEAD_TO_SEQ, y=o_flat)
+    return x.gather(o_flat)

@@ -137,6 +137,21 @@ def _worker(rank, world, port, case, q):
             el = float(np.abs(lse.numpy() - rl[:, h0:h1]).max()) if h1 > h0 else 0.0
             assert lse.shape == (B, h1 - h0, sum(lens))
             q.put((rank, "ok", eo, el))
+        elif case == "usp_2d":
+            # R = 2 ring ranks x U = 2 Ulysses ranks, rank g = r * U + u holds
+            # sequence shard g; uneven shards everywhere (5, 4, 6, 3 tokens)
+            R, U, B, H, D, lens = 2, 2, 2, 4, 8, [5, 4, 6, 3]
+            uly = [dist.new_group([r * U + u for u in range(U)]) for r in range(R)]
+            ring = [dist.new_group([r * U + u for r in range(R)]) for u in range(U)]
+            r_me, u_me = divmod(rank, U)
+            qa, ka, va = wl.make_qkv(B, H, sum(lens), D, torch.float32, 76)
+            o0 = sum(lens[:rank])
+            sl = slice(o0, o0 + lens[rank])
+            out = cpd.usp_attention_2d(qa[:, sl].contiguous(), ka[:, sl].contiguous(),
+                                       va[:, sl].contiguous(), ring[u_me], uly[r_me], ops=ops)
+            ro, _ = oracle.attention(qa.double().numpy(), ka.double().numpy(),
+                                     va.double().numpy())
+            q.put((rank, "ok", float(np.abs(out.numpy() - ro[:, sl]).max()), 0.0))
         elif case == "rank_leaves":
             # rank 1 leaves between steps without joining the exchange: rank 0's
             # metadata all-gather must end with an error within the group's
@@ -212,6 +227,12 @@ def test_ulysses_anything_uneven_shards_and_heads_over_three_ranks():
     for rank, status, eo, el in _run("ulysses_uneven", world=3):
         assert status == "ok", status
         assert eo <= 1e-5 and el <= 1e-5, (rank, eo, el)
+
+
+def test_unified_2d_mesh_over_four_ranks():
+    for rank, status, eo, _ in _run("usp_2d", world=4):
+        assert status == "ok", status
+        assert eo <= 1e-5, (rank, eo)
 
 
 def test_shape_mismatch_raises_on_every_rank():

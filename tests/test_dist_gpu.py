@@ -57,3 +57,12 @@ def test_ulysses_all_to_all_one_rank(one_rank):
     torch.cuda.synchronize()
     ro, rl = oracle.attention(_np(q), _np(k), _np(v))
     assert np.abs(_np(out) - ro).max() <= 2e-2 and np.abs(_np(lse) - rl).max() <= 1e-3
+
+
+def test_unified_2d_one_rank(one_rank):
+    q, k, v = wl.make_qkv(2, 4, 300, 128, torch.bfloat16, 83)
+    g = dist.group.WORLD
+    out = cpd.usp_attention_2d(q.cuda(), k.cuda(), v.cuda(), g, g, one_rank, one_rank)
+    torch.cuda.synchronize()
+    ro, _ = oracle.attention(_np(q), _np(k), _np(v))
+    assert np.abs(_np(out) - ro).max() <= 2e-2
