@@ -84,6 +84,21 @@ def test_ulysses_permute_into_strided_view(cuda_ok):
 
 
 # ---------------------------------------------------------------- LSE merge
+def test_lse_merge_full_size_flux_shape(cuda_ok):
+    """The merge at the benchmark's shape ([1, 4608, 24, 128] fp32), every
+    element compared with the oracle."""
+    g = torch.Generator().manual_seed(9)
+    shape, lshape = (1, 4608, 24, 128), (1, 24, 4608)
+    oa, oi = torch.randn(shape, generator=g), torch.randn(shape, generator=g)
+    la, li = torch.randn(lshape, generator=g) * 4, torch.randn(lshape, generator=g) * 4
+    ref_o, ref_l = oracle.lse_merge(_np(oa), _np(la), _np(oi), _np(li))
+    da, dla = oa.cuda(), la.cuda()
+    cp.lse_merge(da, dla, oi.cuda(), li.cuda())
+    torch.cuda.synchronize()
+    assert np.abs(_np(da) - ref_o).max() <= 1e-5
+    assert np.abs(_np(dla) - ref_l).max() <= 1e-5
+
+
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("in_dtype", [torch.float32, torch.bfloat16])
 def test_lse_merge(cuda_ok, D, in_dtype):
@@ -374,6 +389,40 @@ def test_workload_hires_outliers_ring8_sampled(cuda_ok):
 
 def test_workload_video_ring_anything8_sampled(cuda_ok):
     _workload_ring("video_ring_anything8", 24, 3)
+
+
+def test_workload_flux_literal_per_chunk_walk_sampled(cuda_ok):
+    """The FLUX ring as the benchmark's per-chunk walk times it: chunk 0
+    with cp_attn_partial, chunks 1-3 folded in with cp_attn_partial_merge."""
+    w = wl.workload("flux_joint_ring4")
+    q, k, v = wl.make_workload_inputs(w)
+    offs = wl.chunk_offsets(wl.ring_chunk_lengths(w.S, w.ring_degree))
+    dq, dk, dv = _dev(q, k, v)
+    out, lse = cp.attn_partial(dq, dk[:, offs[0]:offs[1]], dv[:, offs[0]:offs[1]])
+    for c in range(1, w.ring_degree):
+        cp.attn_partial_merge(dq, dk[:, offs[c]:offs[c + 1]], dv[:, offs[c]:offs[c + 1]], out, lse)
+    torch.cuda.synchronize()
+    rows = _rows(w.S, 64, 11)
+    ro, rl = oracle.attention(_np(q), _np(k), _np(v), rows=rows)
+    _check(out, lse, ro, rl, w.torch_dtype, rows=rows)
+
+
+def test_workload_flux_gathered_uneven_sampled(cuda_ok):
+    """The FLUX keys as the benchmark's Ring Anything component lays them
+    out: shards of 1172, 1172, 1172, 1092 padded to 1172, own chunk first,
+    the three other slots folded in with one gathered launch."""
+    w = wl.workload("flux_joint_ring4")
+    q, k, v = wl.make_workload_inputs(w)
+    lens = [1172, 1172, 1172, 1092]
+    kg = _padded_gather(k, lens, 1172, 0.0).cuda()
+    vg = _padded_gather(v, lens, 1172, 0.0).cuda()
+    dq = q.cuda()
+    out, lse = cp.attn_partial(dq, kg[0, :, :lens[0]], vg[0, :, :lens[0]])
+    cp.ring_attention_gathered(dq, kg, vg, lens, skip_chunk=0, out=out, lse=lse, accumulate=True)
+    torch.cuda.synchronize()
+    rows = _rows(w.S, 64, 12)
+    ro, rl = oracle.attention(_np(q), _np(k), _np(v), rows=rows)
+    _check(out, lse, ro, rl, w.torch_dtype, rows=rows)
 
 
 @pytest.mark.parametrize("R,U", [(1, 4), (2, 2)])
