@@ -492,6 +492,17 @@ def _extra_workloads(cp, wl, dev, stream, flush, tc_peak):
         tf = w.flops / (np.mean(t) * 1e-3) / 1e12
         res[name] = {"ms": float(np.mean(t)), "TFLOP/s": tf, "frac_of_bf16_peak": tf / tc_peak}
         del q, k, v, out, lse
+    # head dim 64: the FLUX token count with twice the heads (same flops)
+    q, k, v = (t.to(dev) for t in wl.make_qkv(1, 48, 4608, 64, torch.bfloat16, 1201, "kscale"))
+    offs = wl.chunk_offsets(wl.ring_chunk_lengths(4608, 4))
+    out = torch.empty((1, 4608, 48, 64), dtype=torch.float32, device=dev)
+    lse = torch.empty((1, 48, 4608), dtype=torch.float32, device=dev)
+    t = _time_loop(lambda: cp.ring_attention(q, k, v, offs, out=out, lse=lse), 20, 3, flush, stream)
+    f64 = 4.0 * 48 * 4608 * 4608 * 64
+    tf = f64 / (np.mean(t) * 1e-3) / 1e12
+    res["ring_d64_h48_s4608_r4"] = {"ms": float(np.mean(t)), "TFLOP/s": tf,
+                                    "frac_of_bf16_peak": tf / tc_peak}
+    del q, k, v, out, lse
     u = wl.workload("ulysses4_unified2x2")
     q, k, v = wl.make_workload_inputs(u)
     for R, U in ((1, 4), (2, 2)):
