@@ -215,10 +215,13 @@ def test_fused_ring_matches_literal_walk(cuda_ok, dtype):
 
 @pytest.mark.parametrize("B,H,Sq,Skv,D,out_dtype", [(3, 2, 300, 200, 128, torch.float32),
                                                     (2, 5, 129, 640, 64, torch.bfloat16),
-                                                    (1, 1, 1000, 3, 128, torch.bfloat16)])
+                                                    (1, 1, 1000, 3, 128, torch.bfloat16),
+                                                    (1, 3, 1, 1, 128, torch.float32),
+                                                    (2, 1, 1, 257, 64, torch.float32)])
 def test_ring_tensor_core_shapes(cuda_ok, B, H, Sq, Skv, D, out_dtype):
     """Batches, S_q != S_kv, a query view whose heads are strided (every other
-    head of a wider tensor), bf16 output, and no lse output."""
+    head of a wider tensor), bf16 output, no lse output, and the smallest
+    cases: one query against one key, one query against a ragged tail."""
     g = torch.Generator().manual_seed(B * 100 + H)
     wide = torch.randn(B, Sq, 2 * H, D, generator=g).bfloat16()
     q = wide[:, :, ::2]                       # head stride 2*D: TMA reads it in place
