@@ -532,3 +532,59 @@ def test_bounded_wait_reports_timeout(cuda_ok):
     out, _ = cp.attn_partial(*_dev(q, k, v))
     torch.cuda.synchronize()
     assert torch.isfinite(out).all()
+
+
+# ---------------------------------------------------------------- seeded random sweep
+def _sweep_cases(n, seed):
+    rng = np.random.default_rng(seed)
+    cases = []
+    for i in range(n):
+        dtype = [torch.bfloat16, torch.float32][int(rng.integers(0, 4) == 0)]
+        D = int(rng.choice([64, 128]))
+        B, H = int(rng.integers(1, 4)), int(rng.integers(1, 5))
+        Sq = int(rng.choice([1, int(rng.integers(2, 129)), int(rng.integers(129, 700))]))
+        R = int(rng.integers(1, 6))
+        cuts = np.sort(rng.integers(0, int(rng.integers(1, 900)) + 1, size=R - 1))
+        Skv = int(cuts[-1]) if R > 1 and rng.random() < 0.3 else int(rng.integers(1, 900))
+        cuts = np.clip(cuts, 0, Skv)
+        offs = [0] + [int(c) for c in cuts] + [Skv]
+        path = ["ring", "walk", "merge_walk", "gathered"][i % 4]
+        cases.append((i, dtype, D, B, H, Sq, offs, path))
+    return cases
+
+
+@pytest.mark.parametrize("case", _sweep_cases(24, 2026), ids=lambda c: f"{c[0]}-{c[7]}")
+def test_seeded_random_sweep(cuda_ok, case):
+    """Random shapes, chunkings (empty chunks included) and call paths, each
+    against one-shot attention."""
+    i, dtype, D, B, H, Sq, offs, path = case
+    Skv = offs[-1]
+    q, k, v = wl.make_qkv(B, H, Sq, D, dtype, 500 + i, "kscale", S_kv=Skv)
+    dq, dk, dv = _dev(q, k, v)
+    R = len(offs) - 1
+    if path == "ring":
+        out, lse = cp.ring_attention(dq, dk, dv, offs)
+    elif path == "walk":
+        out = torch.zeros(B, Sq, H, D, device="cuda")
+        lse = torch.full((B, H, Sq), -float("inf"), device="cuda")
+        for c in range(R):
+            oc, lc = cp.attn_partial(dq, dk[:, offs[c]:offs[c + 1]], dv[:, offs[c]:offs[c + 1]])
+            cp.lse_merge(out, lse, oc, lc)
+    elif path == "merge_walk":
+        out = torch.zeros(B, Sq, H, D, device="cuda")
+        lse = torch.full((B, H, Sq), -float("inf"), device="cuda")
+        for c in reversed(range(R)):
+            cp.attn_partial_merge(dq, dk[:, offs[c]:offs[c + 1]], dv[:, offs[c]:offs[c + 1]],
+                                  out, lse)
+    else:
+        lens = [offs[c + 1] - offs[c] for c in range(R)]
+        L = max(max(lens), 1)
+        kg = _padded_gather(k, lens, L, float("nan")).cuda()
+        vg = _padded_gather(v, lens, L, 0.0).cuda()
+        out, lse = cp.ring_attention_gathered(dq, kg, vg, lens)
+    torch.cuda.synchronize()
+    ro, rl = oracle.attention(_np(q), _np(k), _np(v))
+    if Skv == 0:
+        assert bool((out == 0).all()) and bool(torch.isneginf(lse).all())
+        return
+    _check(out, lse, ro, rl, dtype)
