@@ -2,9 +2,8 @@
 
 Tolerances: fp32 inputs, max-abs 1e-4 on out and lse; bf16 inputs, max-abs
 2e-2 on out and 1e-3 on lse; the Ulysses permutation is compared bit for bit.
-Small cases span several 128-row tiles with ragged tails; the five full-size
-workloads run in the same launch configuration the benchmark times and are
-checked on seeded samples of query rows the oracle computes one by one.
+Small cases span several 128-row tiles with ragged tails.  The five
+full-size workloads are in test_gpu_workloads_full.py.
 """
 import numpy as np
 import pytest
@@ -13,6 +12,7 @@ import torch
 import oracle
 import context_attention_dits_cp_b200 as cp
 from context_attention_dits_cp_b200 import workloads as wl
+from test_gpu_workloads_full import oracle_by_head
 
 pytestmark = pytest.mark.gpu
 
@@ -40,12 +40,6 @@ def _check(out, lse, ref_out, ref_lse, dtype, rows=None):
     assert eo <= tol_o, f"out max-abs {eo:.3e} > {tol_o}"
     assert el <= tol_l, f"lse max-abs {el:.3e} > {tol_l}"
     return eo, el
-
-
-def _rows(S, n, seed):
-    rng = np.random.default_rng(seed)
-    base = np.unique(np.concatenate([[0, S - 1], rng.choice(S, size=min(n, S), replace=False)]))
-    return np.sort(base)
 
 
 # ---------------------------------------------------------------- Ulysses permute
@@ -359,90 +353,7 @@ def test_constant_v_and_zero_q_closed_forms(cuda_ok):
     assert (lse.cpu() - np.log(S)).abs().max().item() <= 1e-3
 
 
-# ---------------------------------------------------------------- full-size workloads
-def _workload_ring(name, n_rows, seed):
-    w = wl.workload(name)
-    q, k, v = wl.make_workload_inputs(w)
-    offs = wl.chunk_offsets(wl.ring_chunk_lengths(w.S, w.ring_degree))
-    out, lse = cp.ring_attention(*_dev(q, k, v), offs)
-    torch.cuda.synchronize()
-    rows = _rows(w.S, n_rows, seed)
-    ro, rl = oracle.attention(_np(q), _np(k), _np(v), rows=rows)
-    return _check(out, lse, ro, rl, w.torch_dtype, rows=rows)
-
-
-def test_workload_tiny_ring_f32_full(cuda_ok):
-    w = wl.workload("tiny_ring_f32")
-    q, k, v = wl.make_workload_inputs(w)
-    offs = wl.chunk_offsets(wl.ring_chunk_lengths(w.S, w.ring_degree))
-    assert offs == [0, 128, 256]
-    out, lse = cp.ring_attention(*_dev(q, k, v), offs)
-    torch.cuda.synchronize()
-    ro, rl = oracle.attention(_np(q), _np(k), _np(v))
-    _check(out, lse, ro, rl, torch.float32)
-
-
-def test_workload_flux_ring4_sampled(cuda_ok):
-    _workload_ring("flux_joint_ring4", 96, 1)
-
-
-def test_workload_hires_outliers_ring8_sampled(cuda_ok):
-    _workload_ring("hires_dit_ring8", 48, 2)
-
-
-def test_workload_video_ring_anything8_sampled(cuda_ok):
-    _workload_ring("video_ring_anything8", 24, 3)
-
-
-def test_workload_flux_literal_per_chunk_walk_sampled(cuda_ok):
-    """The FLUX ring as the benchmark's per-chunk walk times it: chunk 0
-    with cp_attn_partial, chunks 1-3 folded in with cp_attn_partial_merge."""
-    w = wl.workload("flux_joint_ring4")
-    q, k, v = wl.make_workload_inputs(w)
-    offs = wl.chunk_offsets(wl.ring_chunk_lengths(w.S, w.ring_degree))
-    dq, dk, dv = _dev(q, k, v)
-    out, lse = cp.attn_partial(dq, dk[:, offs[0]:offs[1]], dv[:, offs[0]:offs[1]])
-    for c in range(1, w.ring_degree):
-        cp.attn_partial_merge(dq, dk[:, offs[c]:offs[c + 1]], dv[:, offs[c]:offs[c + 1]], out, lse)
-    torch.cuda.synchronize()
-    rows = _rows(w.S, 64, 11)
-    ro, rl = oracle.attention(_np(q), _np(k), _np(v), rows=rows)
-    _check(out, lse, ro, rl, w.torch_dtype, rows=rows)
-
-
-def test_workload_flux_gathered_uneven_sampled(cuda_ok):
-    """The FLUX keys as the benchmark's Ring Anything component lays them
-    out: shards of 1172, 1172, 1172, 1092 padded to 1172, own chunk first,
-    the three other slots folded in with one gathered launch."""
-    w = wl.workload("flux_joint_ring4")
-    q, k, v = wl.make_workload_inputs(w)
-    lens = [1172, 1172, 1172, 1092]
-    kg = _padded_gather(k, lens, 1172, 0.0).cuda()
-    vg = _padded_gather(v, lens, 1172, 0.0).cuda()
-    dq = q.cuda()
-    out, lse = cp.attn_partial(dq, kg[0, :, :lens[0]], vg[0, :, :lens[0]])
-    cp.ring_attention_gathered(dq, kg, vg, lens, skip_chunk=0, out=out, lse=lse, accumulate=True)
-    torch.cuda.synchronize()
-    rows = _rows(w.S, 64, 12)
-    ro, rl = oracle.attention(_np(q), _np(k), _np(v), rows=rows)
-    _check(out, lse, ro, rl, w.torch_dtype, rows=rows)
-
-
-@pytest.mark.parametrize("R,U", [(1, 4), (2, 2)])
-def test_workload_ulysses_and_unified_sampled(cuda_ok, R, U):
-    w = wl.workload("ulysses4_unified2x2")
-    q, k, v = wl.make_workload_inputs(w)
-    G = R * U
-    sh = lambda t: wl.sequence_shards(t, G)
-    out, lse = cp.usp_attention(*_dev(sh(q), sh(k), sh(v)), R, U)
-    torch.cuda.synchronize()
-    # back to token order [B, S, H, D]
-    o_full = out.cpu().transpose(0, 1).reshape(w.B, w.S, w.H, w.D)
-    rows = _rows(w.S, 32, 4 + R)
-    ro, rl = oracle.attention(_np(q), _np(k), _np(v), rows=rows)
-    _check(o_full, lse.cpu(), ro, rl, torch.bfloat16, rows=rows)
-
-
+# ---------------------------------------------------------------- unified, small
 @pytest.mark.parametrize("S,D,dtype", [(512, 128, torch.bfloat16),    # shards of 128: fused
                                        (600, 64, torch.bfloat16),     # shards of 150: permute path
                                        (1000, 128, torch.bfloat16),   # shards of 250: permute path
@@ -491,7 +402,7 @@ def test_ulysses_anything_permute_bit_exact(cuda_ok, dtype, B, S, H, D, U):
     assert np.array_equal(bits(x2), bits(x))
 
 
-def test_ulysses_anything_attention_1008px_sampled(cuda_ok):
+def test_ulysses_anything_attention_1008px_every_row(cuda_ok):
     """FLUX at 1008x1008: 3969 image + 512 text tokens on 4 ranks, where the
     guide's plain Ulysses fails and Ulysses Anything runs."""
     B, S, H, D, U = 1, 4481, 24, 128, 4
@@ -501,9 +412,8 @@ def test_ulysses_anything_attention_1008px_sampled(cuda_ok):
                                              B, H, D, so, ho)
     torch.cuda.synchronize()
     o_full = _unflat(out.cpu(), so, B, H, D)
-    rows = _rows(S, 48, 6)
-    ro, rl = oracle.attention(_np(q), _np(k), _np(v), rows=rows)
-    _check(o_full, lse.cpu(), ro, rl, torch.bfloat16, rows=rows)
+    ro, rl = oracle_by_head(_np(q), _np(k), _np(v))     # every row of every head
+    _check(o_full, lse.cpu(), ro, rl, torch.bfloat16)
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
