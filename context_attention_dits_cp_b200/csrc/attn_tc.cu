@@ -381,6 +381,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
         l_run += (a01.x + a01.y) + (a23.x + a23.y);
       }
+      if (t == 0 && valid < kBlockN) {
+        // Ring Anything trim, V side: a chunk's last tile was loaded whole,
+        // and the rows past the chunk end may be padding of any value (a
+        // padded all-gather slot).  Their P is exactly 0, but 0 * NaN is
+        // NaN in the MMA, so the rows are zeroed in shared memory before
+        // P V reads them.  Tile 0's P V is issued first and the slot is not
+        // refilled before both tiles have consumed it.
+        const int n = 2 * j + 1;
+        if (!(ok = mbar_wait(&kv_full[n % NST], (n / NST) & 1, abort_flag, p.err))) break;
+        if (row >= valid) {
+          uint8_t* vrow = sKV + (n % NST) * L::kTileBytes + row * 128;
+#pragma unroll
+          for (int hh = 0; hh < D / 64; ++hh)
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              reinterpret_cast<uint4*>(vrow + hh * L::kHalfBytes)[k] = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();

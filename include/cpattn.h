@@ -161,9 +161,10 @@ int cp_ring_attention(const cp_tensor* q, const cp_tensor* k,
  *               NULL); 1 folds the result into the fp32 accumulator
  *               (out f32, lse required) like cp_attn_partial_merge, and is
  *               a no-op when no chunk remains.
- * The bf16 path reads whole 128-row tiles, so the padding rows of v inside
- * a chunk's last tile are multiplied by exact zeros: they must be finite
- * (zero them when padding).  Padding of k may hold anything.
+ * The padding rows of k and v may hold any value, NaN and Inf included:
+ * the bf16 path loads a chunk's last 128-row tile whole, masks the scores
+ * of the padded keys to -inf and zeroes the padded v rows in shared memory
+ * before P V reads them; the f32 path never loads them.
  */
 int cp_ring_attention_gathered(const cp_tensor* q, const cp_tensor* k_gathered,
                                const cp_tensor* v_gathered,
@@ -231,9 +232,15 @@ size_t cp_usp_workspace_bytes(int64_t B, int64_t S, int64_t H, int64_t D,
  *   - Sizes whose workspace (cp_usp_workspace_bytes) exceeds
  *     CP_USP_STATIC_SCRATCH_BYTES are rejected with CP_ERR_WORKSPACE before
  *     any GPU work.
+ *   - Arguments are checked exactly as by cp_usp_attention and give the
+ *     same error codes.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *     (cudaGetSymbolAddress, with that device current).  With CUDA's lazy
+ *     module loading that lookup also loads this part of the library and
+ *     reserves the array, and it may synchronise the device.  So make one
+ *     call per device before any stream capture or latency-critical hook: a
+ *     call with an empty problem (B = 0) does only this set-up and launches
+ *     nothing.
  *   - Every call shares the one array and it keeps the last call's contents
  *     (all of it is rewritten before it is read, so nothing needs clearing):
  *     calls whose GPU work overlaps -- other streams, other threads -- race.

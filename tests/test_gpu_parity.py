@@ -295,17 +295,19 @@ def _padded_gather(t, lengths, L, pad):
     return g
 
 
+@pytest.mark.parametrize("vpad", [float("nan"), float("inf"), 1e30])
 @pytest.mark.parametrize("dtype,D,B", [(torch.bfloat16, 128, 1), (torch.bfloat16, 64, 2),
                                        (torch.float32, 128, 2)])
-def test_gathered_ring_trims_padding_in_place(cuda_ok, dtype, D, B):
+def test_gathered_ring_trims_padding_in_place(cuda_ok, dtype, D, B, vpad):
     """Ring Anything over a padded all-gather: chunk c is the first
-    lengths[c] rows of slot c; the padding (NaN in K, 1e30 in V) never
-    contributes.  Whole walk, and own chunk first then the rest merged in."""
+    lengths[c] rows of slot c; the padding (NaN in K; NaN, Inf or 1e30 in V)
+    never contributes.  Whole walk, and own chunk first then the rest merged
+    in."""
     lengths, L, H, Sq = [300, 0, 257, 128], 320, 3, 290
     Skv = sum(lengths)
     q, k, v = wl.make_qkv(B, H, Sq, D, dtype, 61, "kscale", S_kv=Skv)
     kg = _padded_gather(k, lengths, L, float("nan")).cuda()
-    vg = _padded_gather(v, lengths, L, 1e30).cuda()
+    vg = _padded_gather(v, lengths, L, vpad).cuda()
     dq = q.cuda()
     ro, rl = oracle.attention(_np(q), _np(k), _np(v))
     out, lse = cp.ring_attention_gathered(dq, kg, vg, lengths)
@@ -490,7 +492,7 @@ def test_seeded_random_sweep(cuda_ok, case):
         lens = [offs[c + 1] - offs[c] for c in range(R)]
         L = max(max(lens), 1)
         kg = _padded_gather(k, lens, L, float("nan")).cuda()
-        vg = _padded_gather(v, lens, L, 0.0).cuda()
+        vg = _padded_gather(v, lens, L, [float("nan"), float("inf")][i % 8 // 4]).cuda()
         out, lse = cp.ring_attention_gathered(dq, kg, vg, lens)
     torch.cuda.synchronize()
     ro, rl = oracle.attention(_np(q), _np(k), _np(v))

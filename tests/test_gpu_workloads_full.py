@@ -108,9 +108,9 @@ def _full_reference(name):
     return _REF[name]
 
 
-def _padded_gather(t, lengths, L):
+def _padded_gather(t, lengths, L, pad):
     B, _, H, D = t.shape
-    g = torch.zeros((len(lengths), B, L, H, D), dtype=t.dtype)
+    g = torch.full((len(lengths), B, L, H, D), pad, dtype=t.dtype)
     o = 0
     for c, n in enumerate(lengths):
         g[c, :, :n] = t[:, o:o + n]
@@ -156,11 +156,12 @@ def test_flux_literal_per_chunk_walk_every_row(cuda_ok):
 def test_flux_gathered_uneven_every_row(cuda_ok):
     """The FLUX keys in Ring Anything shards of 1172, 1172, 1172, 1092 padded
     to 1172: own chunk first from local memory, then the three other slots
-    of the padded all-gather folded in by one gathered launch."""
+    of the padded all-gather folded in by one gathered launch.  The padding
+    holds NaN, which must never reach the result."""
     w, q, k, v = _inputs("flux_joint_ring4")
     lens = [1172, 1172, 1172, 1092]
-    kg = _padded_gather(k, lens, 1172).cuda()
-    vg = _padded_gather(v, lens, 1172).cuda()
+    kg = _padded_gather(k, lens, 1172, float("nan")).cuda()
+    vg = _padded_gather(v, lens, 1172, float("nan")).cuda()
     dq = q.cuda()
     out, lse = cp.attn_partial(dq, kg[0, :, :lens[0]], vg[0, :, :lens[0]])
     cp.ring_attention_gathered(dq, kg, vg, lens, skip_chunk=0, out=out, lse=lse, accumulate=True)
