@@ -9,11 +9,11 @@ K/V, §Ring Anything for uneven shards, §Ulysses Attention):
 * ``ring_attention_allgather`` -- every rank holds its own sequence shard of
   q, k, v, of any length (Ring Anything).  The shard lengths travel over a
   CPU group first, so no device synchronisation is needed for metadata.  Each
-  rank pads K/V to the longest shard (padding zeroed), all-gathers them, and
-  attends its queries to every chunk; the padding is trimmed by the chunk
-  walk itself (``cp_ring_attention_gathered`` reads the gathered slots in
-  place).  The local chunk is folded in from local memory while the
-  all-gather is in flight, so the exchange overlaps that compute.
+  rank pads K/V to the longest shard and the padded shards are exchanged,
+  by default as one asynchronous broadcast per slot: the local chunk is
+  attended while they travel, then each slot's chunk as soon as that slot
+  has landed, while later slots are still in flight.  The padding is
+  trimmed by the chunk extents: no call ever attends it.
 * ``ulysses_attention_all_to_all`` -- every rank holds its tokens of all H
   heads.  The heads are packed into U groups, exchanged with one all-to-all
   so that every rank holds all tokens of its head group, attended, and sent
@@ -69,36 +69,78 @@ def exchange_shard_meta(q: torch.Tensor, k: torch.Tensor, group=None) -> List[Li
 
 
 def ring_attention_allgather(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, group=None,
-                             cpu_group=None, scale: Optional[float] = None, ops=None):
+                             cpu_group=None, scale: Optional[float] = None, ops=None,
+                             pipeline: str = "slots", trace: Optional[list] = None):
     """Attention of this rank's queries to the whole sharded sequence.
 
     q, k, v: this rank's shard [B, s_r, H, D]; s_r may differ across ranks.
     group:   the device group (NCCL) that carries K/V; cpu_group: the group
              that carries the shard lengths (gloo; defaults to ``group``).
+    pipeline:
+      ``"slots"``  (default) the padded all-gather is split into one
+                   broadcast per slot (slot c = rank c's padded [K; V]),
+                   all issued at once and asynchronous.  The local chunk is
+                   attended while they travel; then slot after slot, each
+                   chunk's attention is issued as soon as its own transfer
+                   has completed, folded into the accumulator by
+                   cp_attn_partial_merge, while the later slots are still in
+                   flight (the guide's ring: K/V move while the block in hand
+                   is attended).
+      ``"gather"`` one all-gather of every slot, overlapped with the local
+                   chunk only, then one cp_ring_attention_gathered launch
+                   over all other slots.
+    trace:   optional list; the "slots" pipeline appends ("wait", c) when it
+             makes the compute stream wait for slot c and ("attend", c) when
+             it issues slot c's attention (own chunk included).
     Returns (out [B, s_q, H, D] fp32, lse [B, H, s_q] fp32) for the local
-    queries against all ranks' keys, chunks merged in rank order.
+    queries against all ranks' keys.
     """
     ops = binding if ops is None else ops
+    if pipeline not in ("slots", "gather"):
+        raise ValueError(f"unknown pipeline {pipeline!r}")
     rank = dist.get_rank(group)
     meta = exchange_shard_meta(q, k, cpu_group if cpu_group is not None else group)
     lengths = [m[0] for m in meta]
+    R = len(lengths)
     L = max(lengths)
     B, s, H, D = k.shape
-    # Ring Anything: pad K/V to the longest shard; padding rows are zeroed
-    # (the gathered-ring call needs them finite), then all-gather [K; V].
-    send = torch.empty((2, B, L, H, D), dtype=k.dtype, device=k.device)
-    send[0, :, :s].copy_(k)
-    send[1, :, :s].copy_(v)
-    if s < L:
-        send[:, :, s:].zero_()
-    recv = torch.empty(len(lengths) * send.numel(), dtype=k.dtype, device=k.device)
-    work = dist.all_gather_into_tensor(recv, send.view(-1), group=group, async_op=True)
-    recv = recv.view(len(lengths), 2, B, L, H, D)
-    # the local chunk needs no exchange: fold it in while K/V travel
+    # Ring Anything: pad K/V to the longest shard.  The padding rows are left
+    # as they are: no call below ever attends them, whatever they hold.
+    recv = torch.empty((R, 2, B, L, H, D), dtype=k.dtype, device=k.device)
+    if pipeline == "gather":
+        send = torch.empty((2, B, L, H, D), dtype=k.dtype, device=k.device)
+        send[0, :, :s].copy_(k)
+        send[1, :, :s].copy_(v)
+        work = dist.all_gather_into_tensor(recv.view(-1), send.view(-1), group=group,
+                                           async_op=True)
+        # the local chunk needs no exchange: fold it in while K/V travel
+        out, lse = ops.attn_partial(q, k, v, scale=scale)
+        work.wait()
+        ops.ring_attention_gathered(q, recv[:, 0], recv[:, 1], lengths, skip_chunk=rank,
+                                    scale=scale, out=out, lse=lse, accumulate=True)
+        return out, lse
+    # "slots": every rank issues the same broadcasts in the same (rank)
+    # order; rank c's slot is its own send buffer
+    recv[rank, 0, :, :s].copy_(k)
+    recv[rank, 1, :, :s].copy_(v)
+    works = [dist.broadcast(recv[c], src=dist.get_global_rank(group, c) if group is not None
+                            else c, group=group, async_op=True) for c in range(R)]
+    if trace is not None:
+        trace.append(("attend", rank))
     out, lse = ops.attn_partial(q, k, v, scale=scale)
-    work.wait()
-    ops.ring_attention_gathered(q, recv[:, 0], recv[:, 1], lengths, skip_chunk=rank, scale=scale,
-                                out=out, lse=lse, accumulate=True)
+    for c in range(R):
+        if c == rank:
+            continue
+        if trace is not None:
+            trace.append(("wait", c))
+        works[c].wait()          # the compute stream waits for slot c only
+        if lengths[c] == 0:
+            continue
+        if trace is not None:
+            trace.append(("attend", c))
+        n = lengths[c]
+        ops.attn_partial_merge(q, recv[c, 0, :, :n], recv[c, 1, :, :n], out, lse, scale=scale)
+    works[rank].wait()           # our own broadcast, before recv can be freed
     return out, lse
 
 

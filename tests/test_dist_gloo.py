@@ -42,6 +42,13 @@ class OracleOps:
         out, lse = self.o.attention_partial(self._np(q), self._np(k), self._np(v), scale)
         return torch.from_numpy(out).float(), torch.from_numpy(lse).float()
 
+    def attn_partial_merge(self, q, k, v, out, lse, scale=None):
+        oc, lc = self.o.attention_partial(self._np(q), self._np(k), self._np(v), scale)
+        acc, lacc = self.o.lse_merge(self._np(out), self._np(lse), oc, lc)
+        out.copy_(torch.from_numpy(acc))
+        lse.copy_(torch.from_numpy(lacc))
+        return out, lse
+
     def ring_attention_gathered(self, q, kg, vg, lengths, skip_chunk=-1, scale=None, out=None,
                                 lse=None, accumulate=False):
         assert accumulate and out is not None and lse is not None
@@ -90,20 +97,43 @@ def _worker(rank, world, port, case, q):
         from context_attention_dits_cp_b200 import dist as cpd
         from context_attention_dits_cp_b200 import workloads as wl
         ops = OracleOps(oracle)
-        if case == "ring":
-            # Ring Anything: uneven shards (and an uneven query split)
-            kv_len, q_len, H, D = [37, 29], [20, 33], 3, 16
+        if case in ("ring", "ring3"):
+            # Ring Anything: uneven shards (and an uneven query split); over
+            # three ranks one rank holds no keys at all.  Both exchanges: one
+            # broadcast per slot (pipelined) and one all-gather.
+            if case == "ring":
+                kv_len, q_len, H, D = [37, 29], [20, 33], 3, 16
+            else:
+                kv_len, q_len, H, D = [21, 0, 17], [9, 12, 5], 2, 8
             qa, ka, va = wl.make_qkv(2, H, sum(q_len), D, torch.float32, 71, S_kv=sum(kv_len))
             qo, ko = sum(q_len[:rank]), sum(kv_len[:rank])
             ql = qa[:, qo:qo + q_len[rank]]
             kl = ka[:, ko:ko + kv_len[rank]].contiguous()
             vl = va[:, ko:ko + kv_len[rank]].contiguous()
-            out, lse = cpd.ring_attention_allgather(ql, kl, vl, ops=ops)
             ro, rl = oracle.attention(qa.double().numpy(), ka.double().numpy(),
                                       va.double().numpy())
-            eo = float(np.abs(out.numpy() - ro[:, qo:qo + q_len[rank]]).max())
-            el = float(np.abs(lse.numpy() - rl[:, :, qo:qo + q_len[rank]]).max())
+            eo = el = 0.0
+            for pipeline in ("slots", "gather"):
+                out, lse = cpd.ring_attention_allgather(ql, kl, vl, ops=ops, pipeline=pipeline)
+                eo = max(eo, float(np.abs(out.numpy() - ro[:, qo:qo + q_len[rank]]).max()))
+                el = max(el, float(np.abs(lse.numpy() - rl[:, :, qo:qo + q_len[rank]]).max()))
             q.put((rank, "ok", eo, el))
+        elif case == "ring_order":
+            # the per-slot pipeline's issue order, as this rank sees it
+            trace = []
+            real = dist.broadcast
+
+            def logged(t, src, group=None, async_op=False):
+                trace.append(("issue", src))
+                return real(t, src, group=group, async_op=async_op)
+
+            dist.broadcast = logged
+            qa, ka, va = wl.make_qkv(1, 2, 4 * world, 8, torch.float32, 77)
+            sl = slice(4 * rank, 4 * rank + 4)
+            cpd.ring_attention_allgather(qa[:, sl], ka[:, sl].contiguous(),
+                                         va[:, sl].contiguous(), ops=ops, trace=trace)
+            dist.broadcast = real
+            q.put((rank, "ok", trace, 0.0))
         elif case == "ulysses":
             B, S, H, D = 2, 10, 4, 8
             qa, ka, va = wl.make_qkv(B, H, S, D, torch.float32, 72)
@@ -215,6 +245,26 @@ def test_ring_allgather_uneven_shards_equals_oneshot():
     for rank, status, eo, el in _run("ring"):
         assert status == "ok", status
         assert eo <= 1e-5 and el <= 1e-5, (rank, eo, el)
+
+
+def test_ring_allgather_three_ranks_one_without_keys():
+    for rank, status, eo, el in _run("ring3", world=3):
+        assert status == "ok", status
+        assert eo <= 1e-5 and el <= 1e-5, (rank, eo, el)
+
+
+def test_ring_slot_pipeline_issue_order():
+    """Every slot's broadcast is issued before any attention; then the local
+    chunk is attended, and slot c's attention comes right after the wait for
+    slot c, before the wait for the next slot."""
+    world = 3
+    for rank, status, trace, _ in _run("ring_order", world=world):
+        assert status == "ok", status
+        want = [("issue", c) for c in range(world)] + [("attend", rank)]
+        for c in range(world):
+            if c != rank:
+                want += [("wait", c), ("attend", c)]
+        assert [tuple(e) for e in trace] == want, (rank, trace)
 
 
 def test_ulysses_all_to_all_equals_oneshot():
