@@ -16,6 +16,15 @@ events; W untimed warm-up steps; K timed steps bracketed by a barrier and a
 device synchronise; max over ranks.  N>1 runs one independent replica of
 the workload per GPU (weak scaling, no collective on the data path).
 ``--impl reference`` times the CPU fp64 oracle on the host cores instead.
+
+``--mode sharded`` (under torchrun) runs the method itself across the ranks
+instead of replicas: the workload's sequence is split over the N ranks
+(Ring Anything ceil split) and every step is one call of the multi-rank
+module -- ``--method ring`` (K/V exchanged slot by slot while the chunk in
+hand is attended), ``ulysses`` (all-to-all, attention per head group,
+inverse all-to-all) or ``usp`` (2 x N/2 mesh).  The line then reports the
+whole sequence's FLOPs over the slowest rank's step time ("scaling":
+"strong") and the bytes each rank sends and receives per step.
 """
 from __future__ import annotations
 
@@ -519,6 +528,147 @@ def _extra_workloads(cp, wl, dev, stream, flush, tc_peak):
     return res
 
 
+# ---------------------------------------------------------------- sharded mode
+def sharded_plan(w, world: int, rank: int, method: str) -> dict:
+    """This rank's share of a sharded step: its token range and the bytes it
+    sends and receives per step over the exchange (counted from the tensors
+    the multi-rank module moves)."""
+    from context_attention_dits_cp_b200 import workloads as wl
+    lens = wl.ring_chunk_lengths(w.S, world)
+    off = wl.chunk_offsets(lens)
+    elt = 4 if w.dtype == "f32" else 2
+    s_me = lens[rank]
+    plan = {"tokens": (off[rank], off[rank + 1]), "shard_lengths": lens}
+    if method == "ring":
+        L = max(lens)
+        slot = 2 * w.B * L * w.H * w.D * elt            # padded [K; V] of one rank
+        plan.update(send=slot, recv=(world - 1) * slot)
+    elif method == "ulysses":
+        hoff = wl.chunk_offsets(wl.ring_chunk_lengths(w.H, world))
+        h_me = hoff[rank + 1] - hoff[rank]
+        tok = w.B * w.D
+        # q, k, v scatter: own tokens of the other groups' heads go out, the
+        # other ranks' tokens of this group's heads come in; the fp32 output
+        # takes the reverse path
+        plan.update(send=3 * tok * s_me * (w.H - h_me) * elt + tok * (w.S - s_me) * h_me * 4,
+                    recv=3 * tok * (w.S - s_me) * h_me * elt + tok * s_me * (w.H - h_me) * 4)
+    elif method == "usp":
+        R, U = 2, world // 2
+        r_me, u_me = divmod(rank, U)
+        grp = [lens[r_me * U + u] for u in range(U)]       # this Ulysses group's shards
+        hoff = wl.chunk_offsets(wl.ring_chunk_lengths(w.H, U))
+        h_me = hoff[u_me + 1] - hoff[u_me]
+        tok = w.B * w.D
+        S_u = sum(grp)
+        blocks = [sum(lens[r * U:(r + 1) * U]) for r in range(R)]
+        slot = 2 * w.B * max(blocks) * h_me * w.D * elt
+        plan.update(send=3 * tok * s_me * (w.H - h_me) * elt + tok * (S_u - s_me) * h_me * 4
+                    + slot,
+                    recv=3 * tok * (S_u - s_me) * h_me * elt + tok * s_me * (w.H - h_me) * 4
+                    + (R - 1) * slot)
+    else:
+        raise ValueError(method)
+    return plan
+
+
+def run_sharded(args, ops=None, device=None):
+    """One rank of ``--mode sharded``: every step is one call of the
+    multi-rank module on this rank's shard of the whole sequence."""
+    import torch.distributed as dist
+    from context_attention_dits_cp_b200 import dist as cpd
+    from context_attention_dits_cp_b200 import workloads as wl
+
+    if device is None:
+        rank, world, local, pg = _dist_init(args.gpus)
+        dev = torch.device("cuda", local if world > 1 else 0)
+        if pg is None:                        # one rank: a group of one
+            import datetime
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", "29517")
+            dist.init_process_group("nccl", rank=0, world_size=1,
+                                    timeout=datetime.timedelta(seconds=120), device_id=dev)
+            pg = dist
+    else:                                     # host-logic tests: gloo ranks on the CPU
+        dev, pg = device, dist
+        rank, world = dist.get_rank(), dist.get_world_size()
+    cpu_group = dist.new_group(backend="gloo") if dev.type == "cuda" else None
+    w = wl.workload(args.workload)
+    method = args.method
+    if method == "usp" and world % 2:
+        raise SystemExit("--method usp needs an even number of ranks (2 x N/2 mesh)")
+    plan = sharded_plan(w, world, rank, method)
+    q, k, v = wl.make_workload_inputs(w)
+    t0, t1 = plan["tokens"]
+    q, k, v = (t[:, t0:t1].contiguous().to(dev) for t in (q, k, v))
+    groups = None
+    if method == "usp":
+        R, U = 2, world // 2
+        uly = [dist.new_group([r * U + u for u in range(U)]) for r in range(R)]
+        ring = [dist.new_group([r * U + u for r in range(R)]) for u in range(U)]
+        r_me, u_me = divmod(rank, U)
+        groups = (ring[u_me], uly[r_me])
+        if dev.type == "cuda":
+            ulyc = [dist.new_group([r * U + u for u in range(U)], backend="gloo")
+                    for r in range(R)]
+            ringc = [dist.new_group([r * U + u for r in range(R)], backend="gloo")
+                     for u in range(U)]
+            groups += (ringc[u_me], ulyc[r_me])
+        else:
+            groups += (None, None)
+
+    def step():
+        if method == "ring":
+            return cpd.ring_attention_allgather(q, k, v, cpu_group=cpu_group, ops=ops)
+        if method == "ulysses":
+            return cpd.ulysses_attention_all_to_all(q, k, v, cpu_group=cpu_group, ops=ops)
+        return cpd.usp_attention_2d(q, k, v, groups[0], groups[1], ring_cpu_group=groups[2],
+                                    ulysses_cpu_group=groups[3], ops=ops)
+
+    for _ in range(args.warmup):
+        step()
+    _barrier(pg, dev)
+    if dev.type == "cuda":
+        stream = torch.cuda.current_stream(dev)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            step()
+        b.record(stream)
+        _barrier(pg, dev)
+        local_ms = a.elapsed_time(b)
+    else:
+        tt = time.perf_counter()
+        for _ in range(args.steps):
+            step()
+        _barrier(pg, dev)
+        local_ms = 1e3 * (time.perf_counter() - tt)
+    total_ms = _max_over_ranks(pg, float(local_ms), dev)
+    ms_per_step = total_ms / args.steps
+    value = w.flops / (ms_per_step * 1e-3) / 1e12        # whole sequence, all ranks
+    mine = torch.tensor([float(plan["send"]), float(plan["recv"])], dtype=torch.float64)
+    table = [torch.zeros(2, dtype=torch.float64) for _ in range(world)]
+    dist.all_gather(table, mine, group=cpu_group)      # host integers over gloo
+    line = None
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "mode": "sharded",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "S": w.S, "D": w.D,
+                       "method": method, "shard_lengths": plan["shard_lengths"],
+                       "parallelism": {"ring": f"ring{world}", "ulysses": f"ulysses{world}",
+                                       "usp": f"ring2 x ulysses{world // 2}"}[method]},
+            "exchange_bytes_per_rank": [{"send": int(t[0]), "recv": int(t[1])} for t in table],
+        }
+        print(json.dumps(line), flush=True)
+    if dev.type == "cuda":
+        dist.destroy_process_group()
+    return line
+
+
 # ---------------------------------------------------------------- CPU oracle
 def _cpu_threads():
     try:
@@ -603,6 +753,12 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("cuda", "reference"), default="cuda")
+    ap.add_argument("--mode", choices=("replicas", "sharded"), default="replicas",
+                    help="replicas: one independent copy of the workload per GPU (default); "
+                         "sharded: the sequence split over the ranks, exchanged per step")
+    ap.add_argument("--method", choices=("ring", "ulysses", "usp"), default="ring",
+                    help="sharded mode: which exchange")
+    ap.add_argument("--workload", default=WORKLOAD, help="sharded mode: workload name")
     ap.add_argument("--extra", action="store_true", help="also time the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-run", nargs="?", const="ring", default=None,
@@ -613,6 +769,8 @@ def main():
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.mode == "sharded":
+        run_sharded(args)
     else:
         run_cuda(args)
 
