@@ -347,9 +347,13 @@ size_t cp_usp_workspace_bytes(int64_t B, int64_t S, int64_t H, int64_t D, int in
   return usp_unfused_bytes(B, S, H, D, in_dtype, out_dtype);
 }
 
-int cp_usp_attention(const cp_tensor* qs, const cp_tensor* ks, const cp_tensor* vs,
-                     int ring_degree, int ulysses_degree, float scale, void* workspace,
-                     size_t workspace_bytes, cp_tensor* outs, cp_tensor* lse, void* stream) {
+}  // extern "C"
+
+namespace cpattn {
+
+int usp_check_args(const cp_tensor* qs, const cp_tensor* ks, const cp_tensor* vs,
+                   int ring_degree, int ulysses_degree, const cp_tensor* outs,
+                   const cp_tensor* lse) {
   int st;
   if ((st = check_basic(qs, 5)) || (st = check_basic(ks, 5)) || (st = check_basic(vs, 5)) ||
       (st = check_basic(outs, 5)))
@@ -357,15 +361,14 @@ int cp_usp_attention(const cp_tensor* qs, const cp_tensor* ks, const cp_tensor* 
   if (qs->dtype != ks->dtype || qs->dtype != vs->dtype) return CP_ERR_DTYPE;
   const int64_t R = ring_degree, U = ulysses_degree;
   if (R < 1 || U < 1 || R * U > 4096) return CP_ERR_DEGREE;
-  const int64_t G = qs->shape[0], B = qs->shape[1], Sg = qs->shape[2], H = qs->shape[3],
-                D = qs->shape[4];
+  const int64_t G = qs->shape[0], B = qs->shape[1], Sg = qs->shape[2], H = qs->shape[3];
   const cp_tensor* others[3] = {ks, vs, outs};
   for (const cp_tensor* t : others)
     for (int i = 0; i < 5; ++i)
       if (t->shape[i] != qs->shape[i]) return CP_ERR_SHAPE;
   if (G != R * U) return CP_ERR_DEGREE;
   if (H % U) return CP_ERR_DEGREE;
-  const int64_t S = Sg * G, SR = Sg * U, Hg = H / U;
+  const int64_t S = Sg * G;
   if (lse) {
     if ((st = check_basic(lse, 3))) return st;
     if (lse->dtype != CP_F32) return CP_ERR_DTYPE;
@@ -373,6 +376,22 @@ int cp_usp_attention(const cp_tensor* qs, const cp_tensor* ks, const cp_tensor* 
   }
   if (R > CP_MAX_CHUNKS) return CP_ERR_DEGREE;
   if (self_overlapping(outs) || (lse && self_overlapping(lse))) return CP_ERR_ALIAS;
+  return CP_OK;
+}
+
+}  // namespace cpattn
+
+extern "C" {
+
+int cp_usp_attention(const cp_tensor* qs, const cp_tensor* ks, const cp_tensor* vs,
+                     int ring_degree, int ulysses_degree, float scale, void* workspace,
+                     size_t workspace_bytes, cp_tensor* outs, cp_tensor* lse, void* stream) {
+  int st;
+  if ((st = usp_check_args(qs, ks, vs, ring_degree, ulysses_degree, outs, lse))) return st;
+  const int64_t R = ring_degree, U = ulysses_degree;
+  const int64_t G = qs->shape[0], B = qs->shape[1], Sg = qs->shape[2], H = qs->shape[3],
+                D = qs->shape[4];
+  const int64_t S = Sg * G, SR = Sg * U, Hg = H / U;
   if (B == 0 || S == 0 || H == 0) return CP_OK;
 
   // Fused: attention reads q/k/v and writes out in the shard layout through

@@ -57,4 +57,10 @@ int launch_ulysses_anything_permute(const TensorView& x, const TensorView& y, in
                                     const int64_t* head_off, int dir, cudaStream_t stream);
 int launch_wait_timeout_selftest(int spin_limit, int* dev_err, cudaStream_t stream);
 
+// Argument checks of cp_usp_attention (everything but the workspace), shared
+// with cp_usp_attention_static so both report the same error codes.
+int usp_check_args(const cp_tensor* qs, const cp_tensor* ks, const cp_tensor* vs,
+                   int ring_degree, int ulysses_degree, const cp_tensor* outs,
+                   const cp_tensor* lse);
+
 }  // namespace cpattn

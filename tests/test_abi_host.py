@@ -223,6 +223,23 @@ def test_static_scratch_entry_rejects_oversize_before_any_launch():
     assert L.cp_usp_attention_static(None, r(k), r(v), 2, 2, 0.0, r(o), None, None) == -1
 
 
+def test_static_scratch_entry_reports_the_same_errors_as_the_workspace_call():
+    """Argument errors come back with the codes cp_usp_attention gives,
+    before the size check reads anything (all checked on the host)."""
+    L = bd.lib()
+    r = ctypes.byref
+    s = lambda off, dt=bd.CP_BF16: _t([4, 1, 2050, 24, 128], dt, FAKE + off)
+    q, k, v, o = s(0), s(1 << 30), s(2 << 30), s(3 << 30, bd.CP_F32)
+    bad_dt = _t([4, 1, 2050, 24, 128], 7, FAKE + (3 << 30))
+    cases = [((r(q), r(k), r(v), 3, 2, 0.0), r(o)),          # G != R * U
+             ((r(q), r(k), r(v), 2, 2, 0.0), r(bad_dt)),     # unknown output dtype
+             ((r(q), r(k), r(v), 0, 4, 0.0), r(o))]          # ring degree 0
+    for args, out in cases:
+        want = L.cp_usp_attention(*args, None, 0, out, None, None)
+        assert want in (-2, -6)
+        assert L.cp_usp_attention_static(*args, out, None, None) == want
+
+
 def test_ulysses_anything_argument_errors():
     L = bd.lib()
     r = ctypes.byref
