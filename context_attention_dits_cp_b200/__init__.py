@@ -9,6 +9,7 @@ from .binding import (  # noqa: F401
     CpError, attn_partial, attn_partial_merge, lse_merge, ring_attention, ring_attention_gathered,
     ring_chunk_offsets, ulysses_permute,
     usp_attention, usp_workspace_bytes, last_device_error, selftest_wait_timeout,
+    selftest_bounds_check, is_debug_build,
     ulysses_anything_permute, ulysses_anything_attention,
     attention_flops, SEQ_TO_HEAD, HEAD_TO_SEQ,
 )

@@ -16,7 +16,13 @@ from typing import Optional, Sequence
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libcpattn.so")
+# CPATTN_DEBUG=1 selects the bounds-checking build (libcpattn_debug.so,
+# compiled with CP_DEBUG): same entry points, every device-side index checked
+# against its tensor's extent, failures reported as CP_ERR_BOUNDS by
+# cp_last_device_error.
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                         "libcpattn_debug.so" if os.environ.get("CPATTN_DEBUG") == "1"
+                         else "libcpattn.so")
 
 CP_F32, CP_BF16 = 0, 1
 MAX_DIMS = 6
@@ -26,13 +32,14 @@ SEQ_TO_HEAD, HEAD_TO_SEQ = 0, 1
 STATUS = {
     0: "CP_OK", -1: "CP_ERR_NULL", -2: "CP_ERR_DTYPE", -3: "CP_ERR_SHAPE", -4: "CP_ERR_ALIGN",
     -5: "CP_ERR_OFFSETS", -6: "CP_ERR_DEGREE", -7: "CP_ERR_CUDA", -8: "CP_ERR_TIMEOUT",
-    -9: "CP_ERR_WORKSPACE", -10: "CP_ERR_ALIAS",
+    -9: "CP_ERR_WORKSPACE", -10: "CP_ERR_ALIAS", -11: "CP_ERR_BOUNDS",
 }
 EXPORTS = ("cp_attn_partial", "cp_attn_partial_merge", "cp_lse_merge", "cp_ring_attention_gathered", "cp_ring_attention", "cp_ulysses_permute",
            "cp_usp_attention", "cp_usp_attention_static", "cp_usp_workspace_bytes",
            "cp_ulysses_anything_permute", "cp_ulysses_anything_attention",
            "cp_ulysses_anything_workspace_bytes", "cp_ring_chunk_offsets",
-           "cp_status_string", "cp_last_device_error", "cp_selftest_wait_timeout")
+           "cp_status_string", "cp_last_device_error", "cp_selftest_wait_timeout",
+           "cp_selftest_bounds_check")
 
 
 class CpTensor(ctypes.Structure):
@@ -83,6 +90,7 @@ def lib() -> ctypes.CDLL:
         L.cp_status_string.restype = ctypes.c_char_p
         L.cp_last_device_error.argtypes = [vp]
         L.cp_selftest_wait_timeout.argtypes = [i32, vp]
+        L.cp_selftest_bounds_check.argtypes = [vp]
         for n in EXPORTS:
             if n not in ("cp_usp_workspace_bytes", "cp_status_string",
                          "cp_ulysses_anything_workspace_bytes"):
@@ -306,7 +314,8 @@ def usp_attention_static(q_shards, k_shards, v_shards, ring_degree: int, ulysses
 
 
 def last_device_error(device=None) -> int:
-    """Synchronises the current stream; CP_ERR_TIMEOUT if a bounded wait gave up."""
+    """Synchronises the current stream; CP_ERR_TIMEOUT if a bounded wait gave
+    up, CP_ERR_BOUNDS if a debug-build bounds check failed."""
     dev = torch.device("cuda") if device is None else device
     return int(lib().cp_last_device_error(_stream(dev)))
 
@@ -316,6 +325,20 @@ def selftest_wait_timeout(spin_limit: int = 4096, device=None) -> int:
     st = int(lib().cp_selftest_wait_timeout(int(spin_limit), _stream(dev)))
     _check(st, "cp_selftest_wait_timeout")
     return last_device_error(dev)
+
+
+def selftest_bounds_check(device=None) -> int:
+    """One deliberately failing device-side bounds check; returns what
+    cp_last_device_error reports afterwards (CP_ERR_BOUNDS on the debug
+    build, CP_OK on the release build)."""
+    dev = torch.device("cuda") if device is None else device
+    _check(int(lib().cp_selftest_bounds_check(_stream(dev))), "cp_selftest_bounds_check")
+    return last_device_error(dev)
+
+
+def is_debug_build() -> bool:
+    """True when the bounds-checking library (CPATTN_DEBUG=1) is loaded."""
+    return os.path.basename(_LIB_PATH) == "libcpattn_debug.so"
 
 
 def attention_flops(B, H, S_q, S_kv, D) -> float:

@@ -3,7 +3,9 @@
     python -m context_attention_dits_cp_b200.build [--force]
 
 Each .cu file under csrc/ is compiled to an object in _build/ (in parallel)
-and the objects are linked into context_attention_dits_cp_b200/libcpattn.so.
+and the objects are linked into context_attention_dits_cp_b200/libcpattn.so;
+the same sources compiled with -DCP_DEBUG (device-side bounds checks) give
+libcpattn_debug.so.
 The CUDA runtime is linked statically; the driver is reached through
 cudaGetDriverEntryPoint, so nothing links against libcuda directly.
 """
@@ -22,6 +24,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libcpattn.so")
+DEBUG_LIB = os.path.join(PKG, "libcpattn_debug.so")   # CP_DEBUG: device-side bounds checks
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
@@ -44,15 +47,15 @@ def _deps():
                         if f.endswith((".cuh", ".h"))] + [os.path.join(INCLUDE, "cpattn.h")]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(d) <= t for d in _deps())
 
 
-def _compile(src: str, extra) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+def _compile(src: str, extra, tag: str = "") -> str:
+    obj = os.path.join(BUILD, os.path.basename(src) + tag + ".o")
     cmd = [nvcc()] + ARCH + FLAGS + list(extra) + ["-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
@@ -60,20 +63,28 @@ def _compile(src: str, extra) -> str:
     return obj
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and up_to_date():
-        return LIB
+def _build_one(lib: str, extra, tag: str, verbose: bool) -> str:
     os.makedirs(BUILD, exist_ok=True)
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, extra), sources()))
-    tmp = LIB + ".tmp"
+        objs = list(ex.map(lambda s: _compile(s, extra, tag), sources()))
+    tmp = lib + ".tmp"
     cmd = [nvcc()] + ARCH + ["-shared", "-Xcompiler", "-fPIC", "-o", tmp] + objs
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
     if verbose:
-        print(f"built {LIB}")
+        print(f"built {lib}")
+    return lib
+
+
+def build(force: bool = False, verbose: bool = False, extra=(), debug: bool = True) -> str:
+    """Builds libcpattn.so and, with debug=True, the bounds-checking
+    libcpattn_debug.so (same sources compiled with -DCP_DEBUG)."""
+    if force or not up_to_date(LIB):
+        _build_one(LIB, extra, "", verbose)
+    if debug and (force or not up_to_date(DEBUG_LIB)):
+        _build_one(DEBUG_LIB, list(extra) + ["-DCP_DEBUG"], ".debug", verbose)
     return LIB
 
 

@@ -183,7 +183,7 @@ int run_attention(RingArgs& a, cudaStream_t stream) {
     const int64_t len = (a.chunk_end ? a.chunk_end[c] : a.chunk_off[c + 1]) - a.chunk_off[c];
     if (len > 0) total += len;
   }
-  if (total == 0) return a.merge ? CP_OK : launch_fill_empty(a.out, a.lse, stream);
+  if (total == 0) return a.merge ? CP_OK : launch_fill_empty(a.out, a.lse, a.dev_err, stream);
   if (a.q.dtype == CP_BF16) return launch_attn_ring_tc(a, stream);
   return launch_attn_ring_f32(a, stream);
 }
@@ -278,7 +278,9 @@ int cp_lse_merge(cp_tensor* out_acc, cp_tensor* lse_acc, const cp_tensor* out_i,
       overlaps(vla, vli))
     return CP_ERR_ALIAS;
   if (B == 0 || S == 0 || H == 0) return CP_OK;
-  return launch_lse_merge(va, vla, vi, vli, as_stream(stream));
+  int* err = device_error_ptr();
+  if (!err) return CP_ERR_CUDA;
+  return launch_lse_merge(va, vla, vi, vli, err, as_stream(stream));
 }
 
 int cp_ring_attention_gathered(const cp_tensor* q, const cp_tensor* k_gathered,
@@ -334,7 +336,9 @@ int cp_ulysses_permute(const cp_tensor* x, cp_tensor* y, int degree, int dir, vo
   }
   const TensorView vx = view_of(x), vy = view_of(y);
   if (self_overlapping(y) || overlaps(vx, vy)) return CP_ERR_ALIAS;
-  return launch_ulysses_permute(vx, vy, degree, dir, as_stream(stream));
+  int* err = device_error_ptr();
+  if (!err) return CP_ERR_CUDA;
+  return launch_ulysses_permute(vx, vy, degree, dir, err, as_stream(stream));
 }
 
 size_t cp_usp_workspace_bytes(int64_t B, int64_t S, int64_t H, int64_t D, int in_dtype,
@@ -558,8 +562,10 @@ int cp_ulysses_anything_permute(const cp_tensor* x, cp_tensor* y, int64_t B, int
   const TensorView vx = view_of(x), vy = view_of(y);
   if (overlaps(vx, vy)) return CP_ERR_ALIAS;
   if (n == 0) return CP_OK;
+  int* err = device_error_ptr();
+  if (!err) return CP_ERR_CUDA;
   return launch_ulysses_anything_permute(vx, vy, B, H, D, degree, seq_offsets, head_offsets, dir,
-                                         as_stream(stream));
+                                         err, as_stream(stream));
 }
 
 size_t cp_ulysses_anything_workspace_bytes(int64_t B, int64_t S, int64_t H, int64_t D,
@@ -678,6 +684,7 @@ const char* cp_status_string(int status) {
     case CP_ERR_TIMEOUT: return "a bounded device-side wait gave up";
     case CP_ERR_WORKSPACE: return "workspace missing or too small";
     case CP_ERR_ALIAS: return "output overlaps an input";
+    case CP_ERR_BOUNDS: return "a device-side bounds check failed (debug build)";
     default: return "unknown status";
   }
 }
@@ -695,9 +702,15 @@ int cp_last_device_error(void* stream) {
     if (cudaMemcpyAsync(p, &zero, sizeof(int), cudaMemcpyHostToDevice, s) != cudaSuccess)
       return CP_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return CP_ERR_CUDA;
-    return CP_ERR_TIMEOUT;
+    return h == kDevErrBounds ? CP_ERR_BOUNDS : CP_ERR_TIMEOUT;
   }
   return CP_OK;
+}
+
+int cp_selftest_bounds_check(void* stream) {
+  int* p = device_error_ptr();
+  if (!p) return CP_ERR_CUDA;
+  return launch_bounds_selftest(p, as_stream(stream));
 }
 
 int cp_selftest_wait_timeout(int spin_limit, void* stream) {
@@ -724,6 +737,22 @@ __global__ void wait_timeout_selftest_kernel(int spin_limit, int* err) {
   if (threadIdx.x == 0) mbar_wait_polls(&bar, 0, (uint32_t)spin_limit, err);
 }
 }  // namespace
+
+namespace {
+// One deliberately failing bounds check: a debug build records it in the
+// device error word, a release build compiles the check away.  The guarded
+// store only touches this block's own shared memory in either build.
+__global__ void bounds_selftest_kernel(int* err) {
+  __shared__ volatile int cell;
+  const int idx = 1 + (int)threadIdx.x;   // "one past the end" of a 1-element range
+  if (CP_IN_BOUNDS(idx < 1, err)) cell = idx;
+}
+}  // namespace
+
+int launch_bounds_selftest(int* dev_err, cudaStream_t stream) {
+  bounds_selftest_kernel<<<1, 1, 0, stream>>>(dev_err);
+  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
 
 int launch_wait_timeout_selftest(int spin_limit, int* dev_err, cudaStream_t stream) {
   wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(spin_limit, dev_err);

@@ -42,6 +42,8 @@ struct F32Params {
   long long l_sb, l_sh, l_ss;
   int B, H, S_q, n_row_blocks, n_chunks;
   float scale;
+  int* err;
+  long long span_q, span_k, span_v, span_out, span_lse;   // elements (bounds checks)
   int chunk_off[CP_MAX_CHUNKS + 1];   // chunk c covers key tokens [chunk_off[c], chunk_end[c])
   int chunk_end[CP_MAX_CHUNKS];
 };
@@ -73,7 +75,8 @@ __global__ void __launch_bounds__(128) attn_ring_f32_kernel(const __grid_constan
 
   for (int i = threadIdx.x; i < kRowsPerBlock * D; i += blockDim.x) {
     const int r = i / D, d = i % D, s = r0 + r;
-    sQ[r][d] = s < p.S_q ? p.q[b * p.q_sb + (long long)s * p.q_ss + h * p.q_sh + d] : 0.f;
+    const long long off = b * p.q_sb + (long long)s * p.q_ss + h * p.q_sh + d;
+    sQ[r][d] = s < p.S_q && CP_IN_BOUNDS(off >= 0 && off < p.span_q, p.err) ? p.q[off] : 0.f;
   }
 
   float m[kRowsPerWarp], l[kRowsPerWarp], acc[kRowsPerWarp][NV];
@@ -94,8 +97,10 @@ __global__ void __launch_bounds__(128) attn_ring_f32_kernel(const __grid_constan
         const int j = i / D, d = i % D;
         const int key = t0 + j;
         const long long row = key % p.seg_kv, slot = key / p.seg_kv;
-        sK[j][d] = p.k[b * p.k_sb + row * p.k_ss + slot * p.k_sg + h * p.k_sh + d];
-        sV[j][d] = p.v[b * p.v_sb + row * p.v_ss + slot * p.v_sg + h * p.v_sh + d];
+        const long long ok_ = b * p.k_sb + row * p.k_ss + slot * p.k_sg + h * p.k_sh + d;
+        const long long ov_ = b * p.v_sb + row * p.v_ss + slot * p.v_sg + h * p.v_sh + d;
+        sK[j][d] = CP_IN_BOUNDS(ok_ >= 0 && ok_ < p.span_k, p.err) ? p.k[ok_] : 0.f;
+        sV[j][d] = CP_IN_BOUNDS(ov_ >= 0 && ov_ < p.span_v, p.err) ? p.v[ov_] : 0.f;
       }
       __syncthreads();
 #pragma unroll
@@ -131,10 +136,15 @@ __global__ void __launch_bounds__(128) attn_ring_f32_kernel(const __grid_constan
     float o_w = 1.f / l[r];
     const float lse_c = m[r] + logf(l[r]);
     const long long base = b * p.o_sb + (long long)s * p.o_ss + h * p.o_sh;
-    float* lse_p = p.lse != nullptr ? p.lse + b * p.l_sb + h * p.l_sh + (long long)s * p.l_ss
-                                    : nullptr;
+    const long long l_off = b * p.l_sb + h * p.l_sh + (long long)s * p.l_ss;
+    float* lse_p = p.lse != nullptr && CP_IN_BOUNDS(l_off >= 0 && l_off < p.span_lse, p.err)
+                       ? p.lse + l_off
+                       : nullptr;
+    // every lane writes D/32 elements of the row, the last at base + D - 1
+    if (!CP_IN_BOUNDS(base >= 0 && base + D <= p.span_out, p.err)) continue;
     if (p.merge) {
       // fp32 log-sum-exp merge with the accumulator already in (out, lse)
+      if (lse_p == nullptr) continue;
       const float a = *lse_p;
       const float nl = a == -INFINITY ? lse_c
                                       : fmaxf(a, lse_c) + log1pf(expf(-fabsf(a - lse_c)));
@@ -163,7 +173,8 @@ __global__ void __launch_bounds__(128) attn_ring_f32_kernel(const __grid_constan
 // out = 0, lse = -inf: the result of attending to no keys at all.
 __global__ void fill_empty_kernel(void* out, int out_bf16, long long o_sb, long long o_ss,
                                   long long o_sh, float* lse, long long l_sb, long long l_sh,
-                                  long long l_ss, int B, int S, int H, int D) {
+                                  long long l_ss, int B, int S, int H, int D, int* err,
+                                  long long span_o, long long span_l) {
   const long long n = (long long)B * S * H * D;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
        i += (long long)gridDim.x * blockDim.x) {
@@ -174,11 +185,13 @@ __global__ void fill_empty_kernel(void* out, int out_bf16, long long o_sb, long 
     const int s = (int)(r % S);
     const int b = (int)(r / S);
     const long long o = b * o_sb + s * o_ss + h * o_sh + d;
+    if (!CP_IN_BOUNDS(o >= 0 && o < span_o, err)) continue;
     if (out_bf16)
       reinterpret_cast<__nv_bfloat16*>(out)[o] = __float2bfloat16_rn(0.f);
     else
       reinterpret_cast<float*>(out)[o] = 0.f;
-    if (d == 0 && lse != nullptr) lse[b * l_sb + h * l_sh + s * l_ss] = -INFINITY;
+    const long long lo = b * l_sb + h * l_sh + s * l_ss;
+    if (d == 0 && lse != nullptr && CP_IN_BOUNDS(lo >= 0 && lo < span_l, err)) lse[lo] = -INFINITY;
   }
 }
 
@@ -233,6 +246,12 @@ int launch_attn_ring_f32(const RingArgs& a, cudaStream_t stream) {
   for (int c = 0; c < a.n_chunks; ++c)
     prm.chunk_end[c] = (int)(a.chunk_end ? a.chunk_end[c] : a.chunk_off[c + 1]);
   prm.scale = a.scale;
+  prm.err = a.dev_err;
+  prm.span_q = span_elems(a.q);
+  prm.span_k = span_elems(a.k);
+  prm.span_v = span_elems(a.v);
+  prm.span_out = span_elems(a.out);
+  prm.span_lse = span_elems(a.lse);
   const long long grid = (long long)prm.n_row_blocks * prm.H * prm.B;
   if (grid <= 0) return CP_OK;
   if (grid > 0x7fffffffLL) return CP_ERR_SHAPE;
@@ -246,14 +265,16 @@ int launch_attn_ring_f32(const RingArgs& a, cudaStream_t stream) {
   return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
 
-int launch_fill_empty(const TensorView& out, const TensorView& lse, cudaStream_t stream) {
+int launch_fill_empty(const TensorView& out, const TensorView& lse, int* dev_err,
+                      cudaStream_t stream) {
   const long long n = out.shape[0] * out.shape[1] * out.shape[2] * out.shape[3];
   if (n <= 0) return CP_OK;
   const int grid = (int)((n + 255) / 256 < 148 * 16 ? (n + 255) / 256 : 148 * 16);
   fill_empty_kernel<<<grid, 256, 0, stream>>>(
       out.data, out.dtype == CP_BF16, out.stride[0], out.stride[1], out.stride[2],
       static_cast<float*>(lse.data), lse.stride[0], lse.stride[1], lse.stride[2],
-      (int)out.shape[0], (int)out.shape[1], (int)out.shape[2], (int)out.shape[3]);
+      (int)out.shape[0], (int)out.shape[1], (int)out.shape[2], (int)out.shape[3], dev_err,
+      span_elems(out), span_elems(lse));
   return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
 

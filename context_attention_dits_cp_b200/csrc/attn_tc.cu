@@ -89,6 +89,8 @@ struct AttnTcParams {
   int n_q_blocks;                // ceil(S_q / 256)
   int n_tiles;                   // key tiles over all chunks
   int n_chunks;
+  int G_q, G_kv;                 // segments of q and of k/v
+  long long span_lse;            // elements the lse view spans (bounds checks)
   float scale_log2;              // scale * log2(e)
   int chunk_off[CP_MAX_CHUNKS + 1];   // chunk c covers key tokens [chunk_off[c], chunk_end[c])
   int chunk_end[CP_MAX_CHUNKS];
@@ -132,6 +134,9 @@ template <int D, int NST>
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_ring_tc_kernel(const __grid_constant__ AttnTcParams p) {
   using L = TcSmem<D>;
+  // tensor memory: S_0, S_1 (128 columns each), then O_0, O_1 (D each)
+  static_assert(2 * kBlockN + 2 * D <= 512, "tensor memory holds 512 columns");
+  static_assert(L::kTileBytes % (128 * 128) == 0, "staging rounds are whole 128x128-byte boxes");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -195,21 +200,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tma_prefetch_desc(&p.tmap_q);
       tma_prefetch_desc(&p.tmap_k);
       tma_prefetch_desc(&p.tmap_v);
-      mbar_arrive_expect_tx(q_full, 2 * L::kTileBytes);
-      for (int t = 0; t < 2; ++t) {
-        const int r0 = q0 + t * kBlockM;
-        for (int hh = 0; hh < D / 64; ++hh)
-          tma_load_5d(sQ + t * L::kTileBytes + hh * L::kHalfBytes, &p.tmap_q, q_full, hh * 64,
-                      r0 % p.seg_q, h, r0 / p.seg_q, b);
+      bool ok = CP_IN_BOUNDS(q0 < p.S_q && h < p.H && b < p.B, p.err);
+      const bool q_issued = ok;
+      if (ok) {
+        mbar_arrive_expect_tx(q_full, 2 * L::kTileBytes);
+        for (int t = 0; t < 2; ++t) {
+          const int r0 = q0 + t * kBlockM;
+          for (int hh = 0; hh < D / 64; ++hh)
+            tma_load_5d(sQ + t * L::kTileBytes + hh * L::kHalfBytes, &p.tmap_q, q_full,
+                        hh * 64, r0 % p.seg_q, h, r0 / p.seg_q, b);
+        }
+      } else {
+        *abort_flag = 1;
       }
       TileWalk w;
       w.init(p);
-      bool ok = true;
       int n_issued = 0;
-      for (int n = 0; n < 2 * p.n_tiles; ++n) {
+      for (int n = 0; ok && n < 2 * p.n_tiles; ++n) {
         const int slot = n % NST;
         const int use = n / NST;
         if (use > 0 && !mbar_wait(&kv_empty[slot], (use - 1) & 1, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        if (!CP_IN_BOUNDS(w.c < p.n_chunks && w.start >= p.chunk_off[w.c] &&
+                              w.start < p.chunk_end[w.c] && w.start / p.seg_kv < p.G_kv,
+                          p.err)) {
+          *abort_flag = 1;
           ok = false;
           break;
         }
@@ -222,7 +239,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (n & 1) w.next(p);
       }
       // Let every copy this CTA started land before its shared memory goes.
-      mbar_wait_drain(q_full, 0, p.err);
+      if (q_issued) mbar_wait_drain(q_full, 0, p.err);
       if (!ok)
         for (int n = n_issued - NST < 0 ? 0 : n_issued - NST; n < n_issued; ++n)
           mbar_wait_drain(&kv_full[n % NST], (n / NST) & 1, p.err);
@@ -418,8 +435,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const float lse_c = (m_run + log2f(l_run)) * 0.69314718055994530942f;
       float o_w = 1.0f / l_run;   // weight of the raw accumulator O
       float acc_w = 0.f;          // merge mode: weight of the (out, lse) already there
-      float* lse_p = p.lse != nullptr && s_row < p.S_q
-                         ? p.lse + b * p.l_sb + h * p.l_sh + (long long)s_row * p.l_ss
+      const long long l_off = b * p.l_sb + h * p.l_sh + (long long)s_row * p.l_ss;
+      float* lse_p = p.lse != nullptr && s_row < p.S_q &&
+                             CP_IN_BOUNDS(l_off >= 0 && l_off < p.span_lse, p.err)
+                         ? p.lse + l_off
                          : nullptr;
       if (p.merge) {
         // fp32 log-sum-exp merge with the accumulator (ContextParallelConfig
@@ -627,6 +646,9 @@ int launch_attn_ring_tc(const RingArgs& a, cudaStream_t stream) {
   prm.l_sh = a.lse.stride[1];
   prm.l_ss = a.lse.stride[2];
   prm.err = a.dev_err;
+  prm.G_q = a.q.ndim == 5 ? (int)a.q.shape[0] : 1;
+  prm.G_kv = a.k.ndim == 5 ? (int)a.k.shape[0] : 1;
+  prm.span_lse = span_elems(a.lse);
   if (a.q.ndim == 5) {   // [G, B, S/G, H, D] shards, read in place
     prm.B = (int)a.q.shape[1];
     prm.seg_q = (int)a.q.shape[2];

@@ -17,6 +17,25 @@ namespace cpattn {
 // wait that gives up stores kDevErrTimeout there.  cp_last_device_error()
 // reads and clears it.
 constexpr int kDevErrTimeout = 1;
+// A device-side bounds check of a debug build (CP_DEBUG) failed.
+constexpr int kDevErrBounds = 2;
+
+// Record the first device error of a launch sequence: a later error (for
+// example the timeouts that follow an aborted CTA) does not overwrite it.
+__device__ __forceinline__ void raise_dev_err(int* err, int code) { atomicCAS(err, 0, code); }
+
+// Bounds checks of the CP_DEBUG build: CP_IN_BOUNDS(cond, err) is `cond`,
+// and a false condition records kDevErrBounds in the device error word; the
+// caller then skips the access.  Release builds compile it to `true`.
+__device__ __forceinline__ bool bounds_ok(bool cond, int* err) {
+  if (!cond) raise_dev_err(err, kDevErrBounds);
+  return cond;
+}
+#ifdef CP_DEBUG
+#define CP_IN_BOUNDS(cond, err) (::cpattn::bounds_ok((cond), (err)))
+#else
+#define CP_IN_BOUNDS(cond, err) (true)
+#endif
 
 // A wait that has not completed after this many nanoseconds gives up.  No
 // legitimate wait inside one CTA's pipeline lasts longer than milliseconds.
@@ -78,7 +97,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
       if (*abort_flag) return false;
       if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
         *abort_flag = 1;
-        atomicExch(err, kDevErrTimeout);
+        raise_dev_err(err, kDevErrTimeout);
         return false;
       }
     }
@@ -95,7 +114,7 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(a, parity)) return true;
     if ((i & 255u) == 0 && globaltimer_ns() - t0 > kWaitTimeoutNs) {
-      atomicExch(err, kDevErrTimeout);
+      raise_dev_err(err, kDevErrTimeout);
       return false;
     }
   }
@@ -107,7 +126,7 @@ __device__ __forceinline__ bool mbar_wait_polls(uint64_t* bar, uint32_t parity,
   const uint32_t a = smem_u32(bar);
   for (uint32_t i = 0; i < max_polls; ++i)
     if (mbar_try_wait(a, parity)) return true;
-  atomicExch(err, kDevErrTimeout);
+  raise_dev_err(err, kDevErrTimeout);
   return false;
 }
 

@@ -32,6 +32,19 @@ inline TensorView view_of(const cp_tensor* t) {
 
 inline int dtype_size(int dt) { return dt == CP_BF16 ? 2 : 4; }
 
+// Elements from a view's first to its last element, plus one (0 when it is
+// empty or has no data): every valid offset lies in [0, span).  The
+// device-side bounds checks of debug builds test offsets against it.
+inline long long span_elems(const TensorView& t) {
+  if (!t.data) return 0;
+  long long span = 1;
+  for (int i = 0; i < t.ndim; ++i) {
+    if (t.shape[i] == 0) return 0;
+    span += (t.shape[i] - 1) * t.stride[i];
+  }
+  return span;
+}
+
 // Attention over a chunk list (one chunk = cp_attn_partial).
 struct RingArgs {
   TensorView q, k, v;      // [B, S, H, D]; k, v may be [G, B, L, H, D] (token s = row s % L of slot s / L)
@@ -47,15 +60,19 @@ struct RingArgs {
 
 int launch_attn_ring_tc(const RingArgs& a, cudaStream_t stream);    // bf16, tensor cores
 int launch_attn_ring_f32(const RingArgs& a, cudaStream_t stream);   // f32, FFMA
-int launch_fill_empty(const TensorView& out, const TensorView& lse, cudaStream_t stream);
+int launch_fill_empty(const TensorView& out, const TensorView& lse, int* dev_err,
+                      cudaStream_t stream);
 int launch_lse_merge(const TensorView& out_acc, const TensorView& lse_acc,
-                     const TensorView& out_i, const TensorView& lse_i, cudaStream_t stream);
+                     const TensorView& out_i, const TensorView& lse_i, int* dev_err,
+                     cudaStream_t stream);
 int launch_ulysses_permute(const TensorView& x, const TensorView& y, int degree, int dir,
-                           cudaStream_t stream);
+                           int* dev_err, cudaStream_t stream);
 int launch_ulysses_anything_permute(const TensorView& x, const TensorView& y, int64_t B,
                                     int64_t H, int64_t D, int U, const int64_t* seq_off,
-                                    const int64_t* head_off, int dir, cudaStream_t stream);
+                                    const int64_t* head_off, int dir, int* dev_err,
+                                    cudaStream_t stream);
 int launch_wait_timeout_selftest(int spin_limit, int* dev_err, cudaStream_t stream);
+int launch_bounds_selftest(int* dev_err, cudaStream_t stream);
 
 // Argument checks of cp_usp_attention (everything but the workspace), shared
 // with cp_usp_attention_static so both report the same error codes.

@@ -32,6 +32,8 @@ struct MergeParams {
   long long la_sb, la_sh, la_ss;   // lse_acc strides
   long long li_sb, li_sh, li_ss;   // lse_i strides
   int B, S, H, n_sblocks;
+  int* err;
+  long long span_a, span_i, span_la, span_li;   // elements (bounds checks)
 };
 
 template <int V>
@@ -113,14 +115,28 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const __grid_constant__ 
     const int tk = lane & 15;
     if (tk < n_rows) {
       const long long s = s0 + tk;
-      lv = lane < 16 ? __ldcs(p.lse_acc + b * p.la_sb + h * p.la_sh + s * p.la_ss)
-                     : __ldcs(p.lse_i + b * p.li_sb + h * p.li_sh + s * p.li_ss);
+      const long long la = b * p.la_sb + h * p.la_sh + s * p.la_ss;
+      const long long li = b * p.li_sb + h * p.li_sh + s * p.li_ss;
+      if (lane < 16 ? CP_IN_BOUNDS(la >= 0 && la < p.span_la, p.err)
+                    : CP_IN_BOUNDS(li >= 0 && li < p.span_li, p.err))
+        lv = lane < 16 ? __ldcs(p.lse_acc + la) : __ldcs(p.lse_i + li);
     }
   }
   float x[kTok][V], y[kTok][V];
+  // rows whose offsets fail a debug-build bounds check are neither read nor written
+  bool row_ok[kTok];
 #pragma unroll
   for (int t = 0; t < kTok; ++t) {
-    if (t < n_rows) {
+    const long long sr = s0 + t;
+    const long long oa = b * p.a_sb + sr * p.a_ss + h * p.a_sh;
+    const long long oi = b * p.i_sb + sr * p.i_ss + h * p.i_sh;
+    row_ok[t] = t < n_rows && CP_IN_BOUNDS(oa >= 0 && oa + D <= p.span_a && oi >= 0 &&
+                                               oi + D <= p.span_i,
+                                           p.err);
+  }
+#pragma unroll
+  for (int t = 0; t < kTok; ++t) {
+    if (row_ok[t]) {
       const long long sr = s0 + t;
       const FV av = __ldcs(reinterpret_cast<const FV*>(p.acc + b * p.a_sb + sr * p.a_ss +
                                                         h * p.a_sh + lane * V));
@@ -139,13 +155,14 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const __grid_constant__ 
     const float nl = mx + log1pf(expf(-fabsf(a - bb)));
     wa = expf(a - nl);
     wb = expf(bb - nl);
-    __stcs(p.lse_acc + b * p.la_sb + h * p.la_sh + (long long)(s0 + lane) * p.la_ss, nl);
+    const long long la = b * p.la_sb + h * p.la_sh + (long long)(s0 + lane) * p.la_ss;
+    if (CP_IN_BOUNDS(la >= 0 && la < p.span_la, p.err)) __stcs(p.lse_acc + la, nl);
   }
 #pragma unroll
   for (int t = 0; t < kTok; ++t) {
     const float ca = __shfl_sync(0xffffffffu, wa, t);
     const float cb = __shfl_sync(0xffffffffu, wb, t);
-    if (t < n_rows) {
+    if (row_ok[t]) {
       const long long sr = s0 + t;
       float r[V];
 #pragma unroll
@@ -160,8 +177,13 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const __grid_constant__ 
 }  // namespace
 
 int launch_lse_merge(const TensorView& acc, const TensorView& lse_acc, const TensorView& oi,
-                     const TensorView& lse_i, cudaStream_t stream) {
+                     const TensorView& lse_i, int* dev_err, cudaStream_t stream) {
   MergeParams p;
+  p.err = dev_err;
+  p.span_a = span_elems(acc);
+  p.span_i = span_elems(oi);
+  p.span_la = span_elems(lse_acc);
+  p.span_li = span_elems(lse_i);
   p.acc = static_cast<float*>(acc.data);
   p.lse_acc = static_cast<float*>(lse_acc.data);
   p.oi = oi.data;

@@ -32,6 +32,8 @@ struct PermParams {
   int U, B, Sl, Hg;
   int run_words;     // run length in vector words
   int dir;
+  int* err;
+  long long span_x, span_y;   // bytes from the first to one past the last element
 };
 
 template <typename W>
@@ -62,6 +64,11 @@ __global__ void __launch_bounds__(256) ulysses_permute_kernel(const __grid_const
       src = p.x + q * p.xs[0] + b * p.xs[1] + ((long long)pp * p.Sl + s) * p.xs[2];
       dst = p.y + pp * p.ys[0] + b * p.ys[1] + s * p.ys[2] + (long long)q * p.Hg * p.ys[3];
     }
+    const long long run_b = (long long)p.run_words * (long long)sizeof(W);
+    if (!CP_IN_BOUNDS(src >= p.x && src - p.x + run_b <= p.span_x && dst >= p.y &&
+                          dst - p.y + run_b <= p.span_y,
+                      p.err))
+      continue;
     const W* sw = reinterpret_cast<const W*>(src);
     W* dw = reinterpret_cast<W*>(dst);
     for (int w0 = lane; w0 < p.run_words; w0 += 32 * K) {
@@ -90,6 +97,8 @@ struct PermAnyParams {
   long long B, S, H, D;
   long long n_runs;
   int U, dir, es, wbytes;
+  int* err;
+  long long n_elems;          // elements on either side (bounds checks)
   int seq_off[CP_MAX_CHUNKS + 1];
   int head_off[CP_MAX_CHUNKS + 1];
 };
@@ -140,6 +149,9 @@ __global__ void __launch_bounds__(256)
       dst = row * HD + h0 * p.D;
     }
     if (len == 0) continue;
+    if (!CP_IN_BOUNDS(src >= 0 && src + len <= p.n_elems && dst >= 0 && dst + len <= p.n_elems,
+                      p.err))
+      continue;
     const W* sw = reinterpret_cast<const W*>(p.x + src * p.es);
     W* dw = reinterpret_cast<W*>(p.y + dst * p.es);
     const int words = (int)(len * p.es / p.wbytes);
@@ -159,8 +171,11 @@ __global__ void __launch_bounds__(256)
 
 int launch_ulysses_anything_permute(const TensorView& x, const TensorView& y, int64_t B,
                                     int64_t H, int64_t D, int U, const int64_t* seq_off,
-                                    const int64_t* head_off, int dir, cudaStream_t stream) {
+                                    const int64_t* head_off, int dir, int* dev_err,
+                                    cudaStream_t stream) {
   PermAnyParams p;
+  p.err = dev_err;
+  p.n_elems = B * seq_off[U] * H * D;
   p.x = static_cast<const uint8_t*>(x.data);
   p.y = static_cast<uint8_t*>(y.data);
   p.B = B;
@@ -196,9 +211,12 @@ int launch_ulysses_anything_permute(const TensorView& x, const TensorView& y, in
 
 // x, y as validated by the C-ABI: 5-D, same dtype, (heads, D) packed.
 int launch_ulysses_permute(const TensorView& x, const TensorView& y, int U, int dir,
-                           cudaStream_t stream) {
+                           int* dev_err, cudaStream_t stream) {
   const int es = dtype_size(x.dtype);
   PermParams p;
+  p.err = dev_err;
+  p.span_x = span_elems(x) * es;
+  p.span_y = span_elems(y) * es;
   p.x = static_cast<const uint8_t*>(x.data);
   p.y = static_cast<uint8_t*>(y.data);
   for (int i = 0; i < 4; ++i) {

@@ -81,9 +81,11 @@ enum {
   CP_ERR_CUDA = -7,      /* a CUDA runtime/driver call failed               */
   CP_ERR_TIMEOUT = -8,   /* a bounded device-side wait gave up              */
   CP_ERR_WORKSPACE = -9, /* workspace missing or too small                  */
-  CP_ERR_ALIAS = -10     /* an output overlaps an input it must not alias,
+  CP_ERR_ALIAS = -10,    /* an output overlaps an input it must not alias,
                             or maps two of its own elements to one address
                             (a zero stride, or dims that interleave)        */
+  CP_ERR_BOUNDS = -11    /* a device-side bounds check failed (debug build,
+                            libcpattn_debug.so, compiled with CP_DEBUG)     */
 };
 
 /*
@@ -311,8 +313,9 @@ const char* cp_status_string(int status);
 /*
  * cp_last_device_error -- synchronises `stream`, returns CP_ERR_TIMEOUT if a
  * bounded device-side wait in any kernel of this library gave up since the
- * last call (else CP_OK, or CP_ERR_CUDA if the stream reports an error), and
- * clears the flag.
+ * last call, CP_ERR_BOUNDS if a device-side bounds check of the debug build
+ * failed first (else CP_OK, or CP_ERR_CUDA if the stream reports an error),
+ * and clears the flag.
  */
 int cp_last_device_error(void* stream);
 
@@ -324,6 +327,17 @@ int cp_last_device_error(void* stream);
  * hanging or faulting the GPU.
  */
 int cp_selftest_wait_timeout(int spin_limit, void* stream);
+
+/*
+ * cp_selftest_bounds_check -- launches one thread whose single bounds check
+ * fails on purpose (an index one past a one-element range).  The debug build
+ * (libcpattn_debug.so, CP_DEBUG) records it, so the next
+ * cp_last_device_error returns CP_ERR_BOUNDS; the release build compiles the
+ * check away and records nothing.  The guarded store goes to the block's own
+ * shared memory in either build.  Used by the tests to check that the debug
+ * build's checks are live and surface without a GPU fault.
+ */
+int cp_selftest_bounds_check(void* stream);
 
 #ifdef __cplusplus
 }

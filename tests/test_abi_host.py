@@ -28,6 +28,16 @@ def test_library_loads_and_exports_all_symbols():
         assert hasattr(L, name), name
 
 
+def test_debug_library_exports_the_same_symbols():
+    """libcpattn_debug.so (CP_DEBUG: device-side bounds checks) is the same
+    C-ABI: every declared entry point is there."""
+    path = os.path.join(os.path.dirname(bd.__file__), "libcpattn_debug.so")
+    assert os.path.exists(path), "build() makes the debug library too"
+    D = ctypes.CDLL(path)
+    for name in _declared():
+        assert hasattr(D, name), name
+
+
 def _t(shape, dtype=bd.CP_BF16, data=FAKE, strides=None):
     d = bd.CpTensor()
     d.data = data
