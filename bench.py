@@ -92,8 +92,9 @@ class ClockSampler:
              0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
              0x100: "display_clock_setting"}
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, interval_s: float = 0.001):
         self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.interval_s = interval_s
         self._stop = threading.Event()
         self._h = None
         try:
@@ -121,7 +122,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            time.sleep(0.005)
+            time.sleep(self.interval_s)
 
     def __enter__(self):
         if self._h is not None:
@@ -259,7 +260,12 @@ def run_cuda(args):
     for _ in range(args.warmup):
         flush()
         step()
+    # clocks: one sampler inside the timed region, one over everything
+    # measured below as well (e2e and component loops), so that the median
+    # rests on enough samples even when the timed region is a few ms
     sampler = ClockSampler(dev.index)
+    run_sampler = ClockSampler(dev.index)
+    run_sampler.__enter__()
     _barrier(pg, dev)
     with sampler:
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -272,6 +278,7 @@ def run_cuda(args):
         _barrier(pg, dev)
     times = [a.elapsed_time(b) for a, b in evs]
     if args.profile_run:
+        run_sampler.__exit__(None, None, None)
         if rank == 0:
             print(json.dumps({"profile_run": True, "ms_per_step": float(np.mean(times))}))
         if pg is not None:
@@ -455,6 +462,19 @@ def run_cuda(args):
     if args.extra:
         components.update(_extra_workloads(cp, wl, dev, stream, flush, tc_peak))
 
+    run_sampler.__exit__(None, None, None)
+    clocks = sampler.summary()
+    whole = run_sampler.summary()
+    clocks["timed_region_samples"] = clocks.pop("samples", 0)
+    clocks["timed_region_sm_mhz"] = clocks["sm_mhz"]
+    if whole.get("sm_mhz") is not None:
+        # the median over the whole measured run (timed region, e2e and
+        # component loops), the figure the cycle count below uses
+        clocks["sm_mhz"] = whole["sm_mhz"]
+        clocks["samples"] = whole.get("samples", 0)
+        clocks["reasons"] = sorted((set(clocks["reasons"]) - {"unavailable"}) |
+                                   set(whole["reasons"]))
+        clocks["sm_kcycles_per_step"] = ms_per_step * whole["sm_mhz"]
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = _cpu_baseline(q, k, v, w)
@@ -478,7 +498,7 @@ def run_cuda(args):
                     "how": "pinned host q/k/v -> device, cp_ring_attention, out+lse -> "
                            "pinned host, every step; steps pipelined on 3 streams"},
             "gpu_launches": gpu_launches,
-            "clocks": sampler.summary(),
+            "clocks": clocks,
             "components": components,
         }
         if cpu is not None:
