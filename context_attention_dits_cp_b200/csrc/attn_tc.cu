@@ -191,6 +191,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // let the next launch of the stream be scheduled, then wait until the
+  // previous grid has finished and its writes are visible (programmatic
+  // dependent launch; both are no-ops for an ordinary launch)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp < 4) {
    regs_dec<kRegsControl>();
@@ -336,27 +341,41 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int j = 0; j < p.n_tiles; ++j) {
       if (!(ok = mbar_wait(&s_ready[t], j & 1, abort_flag, p.err))) break;
       tc_fence_after();
+      // S in four 32-column chunks: chunk c + 1 is in flight while the row
+      // max of chunk c is taken (eight independent max chains)
       float s[kBlockN];
+      float mx[8];
+      tmem_ld32(tS, s);
+      tmem_wait_ld_into(s);
+      tmem_ld32(tS + 32, s + 32);
 #pragma unroll
-      for (int c = 0; c < kBlockN / 32; ++c) tmem_ld32(tS + c * 32, s + c * 32);
-      tmem_wait_ld();
+      for (int i = 0; i < 8; ++i)
+        mx[i] = max3f(s[4 * i], s[4 * i + 1], fmaxf(s[4 * i + 2], s[4 * i + 3]));
+#pragma unroll
+      for (int c = 1; c < kBlockN / 32; ++c) {
+        tmem_wait_ld_into(s + 32 * c);
+        if (c + 1 < kBlockN / 32) tmem_ld32(tS + 32 * (c + 1), s + 32 * (c + 1));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          mx[i] = max3f(mx[i], s[32 * c + 4 * i], s[32 * c + 4 * i + 1]);
+          mx[i] = max3f(mx[i], s[32 * c + 4 * i + 2], s[32 * c + 4 * i + 3]);
+        }
+      }
       const int valid = w.valid();
       if (valid < kBlockN) {
+        // a chunk's last tile: columns past the chunk end are masked (rare,
+        // so the max is simply taken again over the masked row)
 #pragma unroll
         for (int c = 0; c < kBlockN; ++c)
           if (c >= valid) s[c] = -INFINITY;
-      }
-      float mx[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-      for (int c = 4; c < kBlockN; c += 8) {
-        mx[0] = max3f(mx[0], s[c], s[c + 1]);
-        mx[1] = max3f(mx[1], s[c + 2], s[c + 3]);
-        if (c + 4 < kBlockN) {
-          mx[2] = max3f(mx[2], s[c + 4], s[c + 5]);
-          mx[3] = max3f(mx[3], s[c + 6], s[c + 7]);
-        }
+        for (int i = 0; i < 8; ++i) mx[i] = s[i];
+#pragma unroll
+        for (int c = 8; c < kBlockN; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
       }
-      const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+      const float m_tile =
+          max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
+          sl2;
       {
         // Rescale the rows whose max moved beyond the threshold, then
         // exponentiate on the MUFU unit, which maps the masked -inf columns
@@ -373,7 +392,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int c = 0; c < D / 32; ++c) {
               float o[32];
               tmem_ld32(tO + c * 32, o);
-              tmem_wait_ld();
+              tmem_wait_ld_into(o);
 #pragma unroll
               for (int i = 0; i < 32; ++i) o[i] *= alpha;
               tmem_st32(tO + c * 32, o);
@@ -480,7 +499,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (p.merge) {          // fp32 accumulator: out' = acc_w * out + o_w * O
             float o[32];
             tmem_ld32(tO + bx * 32, o);
-            tmem_wait_ld();
+            tmem_wait_ld_into(o);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
               float4* cell = reinterpret_cast<float4*>(box + ((k ^ (row & 7)) << 4));
@@ -495,7 +514,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int hlf = 0; hlf < 2; ++hlf) {
               float o[32];
               tmem_ld32(tO + bx * 64 + hlf * 32, o);
-              tmem_wait_ld();
+              tmem_wait_ld_into(o);
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
                 uint4 v;
@@ -510,7 +529,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           } else {
             float o[32];
             tmem_ld32(tO + bx * 32, o);
-            tmem_wait_ld();
+            tmem_wait_ld_into(o);
 #pragma unroll
             for (int k = 0; k < 8; ++k)
               *reinterpret_cast<float4*>(box + ((k ^ (row & 7)) << 4)) =
@@ -624,7 +643,20 @@ int launch_tc(const AttnTcParams& prm, int grid, cudaStream_t stream) {
       return CP_ERR_CUDA;
     configured[dev] = true;
   }
-  kern<<<grid, kTcThreads, smem, stream>>>(prm);
+  // Programmatic dependent launch: the kernel may be scheduled while the
+  // previous kernel of the stream drains; it waits for that grid (and its
+  // memory) before touching global memory, so only its set-up overlaps.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, prm) != cudaSuccess) return CP_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
 
