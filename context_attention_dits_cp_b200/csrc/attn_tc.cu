@@ -12,13 +12,26 @@
 // tiles never straddle a chunk boundary; keys past a chunk's end inside its
 // last tile are masked to -inf (that is the Ring Anything trim).
 //
-// CTA = one work unit: two 128-row query tiles of one (batch, head), so each
-// K/V tile brought in by TMA feeds four MMAs.  Warp roles (384 threads):
-//   warp 0      TMA producer: Q once, then K_j, V_j into a ring of NST slots
-//   warp 1      MMA issuer (one thread): S_t = Q_t K^T, O_t += P_t V
+// Work unit = two 128-row query tiles of one (batch, head), so each K/V
+// tile brought in by TMA feeds four MMAs.  The grid is persistent: one CTA
+// per SM walks the units round-robin, and the K/V ring, the barriers and
+// tensor memory carry on from one unit to the next, so the next unit's Q
+// and K/V loads and its first S MMAs overlap the previous unit's last tiles
+// and epilogue.  Warp roles (384 threads):
+//   warp 0      TMA producer: per unit Q (once the previous unit's last S
+//               MMAs have read the Q buffer), then K_j, V_j into a ring of
+//               NST slots
+//   warp 1      MMA issuer (one thread): S_t = Q_t K^T, O_t += P_t V; the
+//               first P V of a unit waits until the previous unit's epilogue
+//               has read O_t out of tensor memory
 //   warp 2      tensor-memory allocator
 //   warps 4-7   softmax + epilogue of query tile 0 (one row per thread)
 //   warps 8-11  softmax + epilogue of query tile 1
+// Epilogue, per warp and its 32 rows: O in rounds of 128 bytes of columns
+// from tensor memory, scaled (or, for the fp32 accumulator, merged with the
+// box the same warp TMA-loads), staged in the warp's own 4 KB of shared
+// memory in the 128-byte swizzled layout and written by one 32-row TMA
+// store; the store's read of the staging area overlaps the next round.
 // Tensor memory (512 columns x 128 lanes x 32 bit):
 //   [0,128)   S_0 (fp32), overwritten in place by P_0 (bf16, 64 columns)
 //   [128,256) S_1 / P_1
@@ -37,6 +50,7 @@
 
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstring>
 
 #include "common.cuh"
@@ -66,9 +80,10 @@ constexpr float kRescaleThreshold = (float)CP_RESCALE_LOG2_THRESHOLD;
 constexpr int kStagesD128 = CP_TC_STAGES_D128;   // 64 KB Q + NST x 32 KB
 constexpr int kStagesD64 = 6;                    // 32 KB Q + NST x 16 KB
 // Register split: the producer/MMA warpgroup gives registers to the two
-// softmax warpgroups (80 + 2 * 208 <= 3 * 168 per thread, the launch budget).
-constexpr int kRegsControl = 80;
-constexpr int kRegsSoftmax = 208;
+// softmax warpgroups (72 + 2 * 216 = 3 * 168 per thread, the launch budget);
+// at this split neither role spills.
+constexpr int kRegsControl = 72;
+constexpr int kRegsSoftmax = 216;
 
 struct AttnTcParams {
   // 5-D maps {D, seg, H, G, B}: token s of the sequence is row s % seg of
@@ -78,6 +93,7 @@ struct AttnTcParams {
   CUtensorMap tmap_k;
   CUtensorMap tmap_v;
   CUtensorMap tmap_out; // box {128 bytes of columns, 128, 1, 1, 1}, 128B swizzle
+  CUtensorMap tmap_out32; // same, 32-row boxes: one warp's rows of one epilogue round
   void* out;
   float* lse;
   int* err;
@@ -90,6 +106,10 @@ struct AttnTcParams {
   int n_tiles;                   // key tiles over all chunks
   int n_chunks;
   int G_q, G_kv;                 // segments of q and of k/v
+  int n_units;                   // work units (2 query tiles of one batch, head)
+  unsigned int* unit_ctr;        // [2]: next unit to hand out, CTAs done (reset by the last)
+  long long o_sg, o_sb, o_ss, o_sh;   // out strides (elements); token s is row s % seg_q
+  long long span_out;            // elements the out view spans (bounds checks)
   long long span_lse;            // elements the lse view spans (bounds checks)
   float scale_log2;              // scale * log2(e)
   int chunk_off[CP_MAX_CHUNKS + 1];   // chunk c covers key tokens [chunk_off[c], chunk_end[c])
@@ -130,43 +150,92 @@ struct TcSmem {
   static constexpr int kHalfBytes = 128 * 64 * 2;  // one 64-column TMA box
 };
 
+// tcgen05 MMAs whose shared-memory descriptors are formed inside the asm
+// statement: the 32-bit low word (start address >> 4 | LBO >> 4 << 16) is a
+// base register plus an immediate, the high word (SBO, version, 128-byte
+// swizzle) an immediate.  The compiler cannot hoist 64-bit descriptors out of
+// the loop, which keeps the issuing thread's register footprint small.
+constexpr uint32_t kDescHi = (uint32_t)((1024u >> 4) | (1u << 14) | (2u << 29));   // bits 32..63
+__device__ __forceinline__ uint32_t desc_lo(uint32_t saddr, uint32_t lbo_bytes) {
+  return ((saddr >> 4) & 0x3FFFu) | ((lbo_bytes >> 4) << 16);
+}
+template <uint32_t AOFF, uint32_t BOFF>
+__device__ __forceinline__ void mma_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b32 al, bl;\n\t.reg .b64 ad, bd;\n\t"
+      "add.u32 al, %1, %5;\n\tadd.u32 bl, %2, %6;\n\t"
+      "mov.b64 ad, {al, %7};\n\tmov.b64 bd, {bl, %7};\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(AOFF), "n"(BOFF), "n"(kDescHi)
+      : "memory");
+}
+template <uint32_t BOFF>
+__device__ __forceinline__ void mma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b32 bl;\n\t.reg .b64 bd;\n\t"
+      "add.u32 bl, %2, %5;\n\tmov.b64 bd, {bl, %6};\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(BOFF), "n"(kDescHi)
+      : "memory");
+}
+
+// Pull a tensor box into L2 (no shared-memory destination, no completion).
+__device__ __forceinline__ void tma_prefetch_l2_5d(const CUtensorMap* map, int c0, int c1,
+                                                   int c2, int c3, int c4) {
+  asm volatile("cp.async.bulk.prefetch.tensor.5d.L2.global [%0, {%1, %2, %3, %4, %5}];" ::"l"(map),
+               "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+               : "memory");
+}
+
+template <int D, int NST>
+struct PersistSmem {
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kStageBytes = 32 * 128;              // per warp: 32 rows x 128 B
+  static constexpr int kStageOff = (2 + NST) * kTileBytes;
+  static constexpr int kBarOff = kStageOff + 8 * kStageBytes;
+  static constexpr size_t kBytes = 1024 + (size_t)kBarOff + 512;
+};
+
 template <int D, int NST>
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_ring_tc_kernel(const __grid_constant__ AttnTcParams p) {
   using L = TcSmem<D>;
-  // tensor memory: S_0, S_1 (128 columns each), then O_0, O_1 (D each)
+  using PS = PersistSmem<D, NST>;
   static_assert(2 * kBlockN + 2 * D <= 512, "tensor memory holds 512 columns");
-  static_assert(L::kTileBytes % (128 * 128) == 0, "staging rounds are whole 128x128-byte boxes");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                                  // 2 tiles
   uint8_t* sKV = smem + 2 * L::kTileBytes;             // NST slots
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NST * L::kTileBytes);
+  uint8_t* sStage = smem + PS::kStageOff;              // 8 warps x 4 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PS::kBarOff);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
+  uint64_t* q_free = bars + 1;          // the unit's last S MMAs are done: Q may be replaced
+  uint64_t* kv_full = bars + 2;
   uint64_t* kv_empty = kv_full + NST;
   uint64_t* s_ready = kv_empty + NST;   // [2]
   uint64_t* p_ready = s_ready + 2;      // [2]
   uint64_t* o_done = p_ready + 2;       // [2]
-  uint64_t* epi_full = o_done + 2;      // [2] a round of staged output is in smem
-  uint64_t* epi_free = epi_full + 2;    // [2] TMA has read the staged round
-  uint64_t* acc_full = epi_free + 2;    // [2] merge mode: the accumulator round is in smem
-  uint64_t* drain = acc_full + 2;       // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* o_free = o_done + 2;        // [2] the epilogue has read O_t out of tensor memory
+  uint64_t* drain = o_free + 2;         // [1]
+  uint64_t* acc_bar = drain + 1;        // [8] merge mode: a warp's accumulator box is in staging
+  uint64_t* unit_full = acc_bar + 8;    // [2] the unit index of slot k & 1 is published
+  uint64_t* unit_free = unit_full + 2;  // [2] every role has read it
+  int* unit_ring_raw = reinterpret_cast<int*>(unit_free + 2);   // [2] published unit indices
+  volatile int* unit_ring = unit_ring_raw;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unit_ring_raw + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int unit = blockIdx.x;
-  const int qblk = unit % p.n_q_blocks;
-  const int hb = unit / p.n_q_blocks;
-  const int h = hb % p.H;
-  const int b = hb / p.H;
-  const int q0 = qblk * 2 * kBlockM;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_free, 1);
     for (int i = 0; i < NST; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
@@ -175,11 +244,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&s_ready[t], 1);
       mbar_init(&p_ready[t], kBlockM / 32);   // one arrive per softmax warp
       mbar_init(&o_done[t], 1);
-      mbar_init(&epi_full[t], kBlockM / 32);   // one arrive per softmax warp
-      mbar_init(&epi_free[t], 1);
-      mbar_init(&acc_full[t], 1);
+      mbar_init(&o_free[t], kBlockM / 32);    // one arrive per softmax warp
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&unit_full[i], 1);
+      mbar_init(&unit_free[i], 1 + 8);   // the MMA thread and the eight softmax warps
+    }
+    for (int i = 0; i < 8; ++i) mbar_init(&acc_bar[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -191,11 +263,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // let the next launch of the stream be scheduled, then wait until the
-  // previous grid has finished and its writes are visible (programmatic
-  // dependent launch; both are no-ops for an ordinary launch)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  // unit u -> (batch, head, first query row); units run round-robin over CTAs
+  auto decode = [&](int u, int& b, int& h, int& q0) {
+    const int qblk = u % p.n_q_blocks;
+    const int hb = u / p.n_q_blocks;
+    h = hb % p.H;
+    b = hb / p.H;
+    q0 = qblk * 2 * kBlockM;
+  };
+  const int tiles2 = 2 * p.n_tiles;   // K/V tile loads per unit
 
   if (warp < 4) {
    regs_dec<kRegsControl>();
@@ -205,9 +284,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tma_prefetch_desc(&p.tmap_q);
       tma_prefetch_desc(&p.tmap_k);
       tma_prefetch_desc(&p.tmap_v);
-      bool ok = CP_IN_BOUNDS(q0 < p.S_q && h < p.H && b < p.B, p.err);
-      const bool q_issued = ok;
-      if (ok) {
+      bool ok = true;
+      int n = 0;          // K/V tile loads issued, over all units
+      int q_loads = 0;
+      for (int k = 0;; ++k) {
+        // the next unit: handed out in index order to whichever CTA asks
+        // first, once this CTA's previous unit no longer needs its Q buffer
+        if (k > 0 && !(ok = mbar_wait(q_free, (k - 1) & 1, abort_flag, p.err))) break;
+        int u = (int)atomicAdd(&p.unit_ctr[0], 1u);
+        if (u >= p.n_units) u = -1;
+        if (k >= 2 && !(ok = mbar_wait(&unit_free[k & 1], ((k >> 1) - 1) & 1, abort_flag, p.err)))
+          break;
+        unit_ring[k & 1] = u;
+        mbar_arrive(&unit_full[k & 1]);
+        if (u < 0) break;
+        int b, h, q0;
+        decode(u, b, h, q0);
+        if (!(ok = CP_IN_BOUNDS(q0 < p.S_q && h < p.H && b < p.B, p.err))) {
+          *abort_flag = 1;
+          break;
+        }
         mbar_arrive_expect_tx(q_full, 2 * L::kTileBytes);
         for (int t = 0; t < 2; ++t) {
           const int r0 = q0 + t * kBlockM;
@@ -215,39 +311,42 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tma_load_5d(sQ + t * L::kTileBytes + hh * L::kHalfBytes, &p.tmap_q, q_full,
                         hh * 64, r0 % p.seg_q, h, r0 / p.seg_q, b);
         }
-      } else {
-        *abort_flag = 1;
+        ++q_loads;
+        TileWalk w;
+        w.init(p);
+        for (int i = 0; i < tiles2; ++i) {
+          const int slot = n % NST;
+          const int use = n / NST;
+          if (use > 0 && !mbar_wait(&kv_empty[slot], (use - 1) & 1, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          if (!CP_IN_BOUNDS(w.c < p.n_chunks && w.start >= p.chunk_off[w.c] &&
+                                w.start < p.chunk_end[w.c] && w.start / p.seg_kv < p.G_kv,
+                            p.err)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&kv_full[slot], L::kTileBytes);
+          const CUtensorMap* m = (i & 1) ? &p.tmap_v : &p.tmap_k;
+          for (int hh = 0; hh < D / 64; ++hh)
+            tma_load_5d(sKV + slot * L::kTileBytes + hh * L::kHalfBytes, m, &kv_full[slot],
+                        hh * 64, w.start % p.seg_kv, h, w.start / p.seg_kv, b);
+          ++n;
+          if (i & 1) w.next(p);
+        }
       }
-      TileWalk w;
-      w.init(p);
-      int n_issued = 0;
-      for (int n = 0; ok && n < 2 * p.n_tiles; ++n) {
-        const int slot = n % NST;
-        const int use = n / NST;
-        if (use > 0 && !mbar_wait(&kv_empty[slot], (use - 1) & 1, abort_flag, p.err)) {
-          ok = false;
-          break;
-        }
-        if (!CP_IN_BOUNDS(w.c < p.n_chunks && w.start >= p.chunk_off[w.c] &&
-                              w.start < p.chunk_end[w.c] && w.start / p.seg_kv < p.G_kv,
-                          p.err)) {
-          *abort_flag = 1;
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&kv_full[slot], L::kTileBytes);
-        const CUtensorMap* m = (n & 1) ? &p.tmap_v : &p.tmap_k;
-        for (int hh = 0; hh < D / 64; ++hh)
-          tma_load_5d(sKV + slot * L::kTileBytes + hh * L::kHalfBytes, m, &kv_full[slot],
-                      hh * 64, w.start % p.seg_kv, h, w.start / p.seg_kv, b);
-        n_issued = n + 1;
-        if (n & 1) w.next(p);
+      // Every fetch of this CTA is done: count it, and the last CTA resets
+      // the counters for the next launch that uses them.
+      if (atomicAdd(&p.unit_ctr[1], 1u) == gridDim.x - 1) {
+        atomicExch(&p.unit_ctr[0], 0u);
+        atomicExch(&p.unit_ctr[1], 0u);
       }
       // Let every copy this CTA started land before its shared memory goes.
-      if (q_issued) mbar_wait_drain(q_full, 0, p.err);
-      if (!ok)
-        for (int n = n_issued - NST < 0 ? 0 : n_issued - NST; n < n_issued; ++n)
-          mbar_wait_drain(&kv_full[n % NST], (n / NST) & 1, p.err);
+      if (q_loads > 0) mbar_wait_drain(q_full, (q_loads - 1) & 1, p.err);
+      for (int i = n - NST < 0 ? 0 : n - NST; i < n; ++i)
+        mbar_wait_drain(&kv_full[i % NST], (i / NST) & 1, p.err);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -256,65 +355,89 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, D, true);
       const uint32_t sQa = smem_u32(sQ);
       const uint32_t sKVa = smem_u32(sKV);
-      // S_t / P_t at columns t*128, O_t at 256 + t*D
-
+      // descriptor low words: start address (16-byte units) | LBO << 16; the
+      // k-steps of one MMA group add compile-time offsets to one base
       auto issue_s = [&](int t, int slot) {
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * L::kHalfBytes + (k & 3) * 32;
-          const uint64_t ad = smem_desc_sw128(sQa + t * L::kTileBytes + off, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sKVa + slot * L::kTileBytes + off, 16, 1024);
-          mma_bf16_ss(tmem + t * 128, ad, bd, idesc_qk, k > 0 ? 1u : 0u);
+        const uint32_t a0 = desc_lo(sQa + t * L::kTileBytes, 16);
+        const uint32_t b0 = desc_lo(sKVa + slot * L::kTileBytes, 16);
+        const uint32_t d = tmem + t * 128;
+        mma_ss_lo<0, 0>(d, a0, b0, idesc_qk, 0u);
+        mma_ss_lo<2, 2>(d, a0, b0, idesc_qk, 1u);
+        mma_ss_lo<4, 4>(d, a0, b0, idesc_qk, 1u);
+        mma_ss_lo<6, 6>(d, a0, b0, idesc_qk, 1u);
+        if constexpr (D == 128) {
+          constexpr uint32_t H = L::kHalfBytes >> 4;
+          mma_ss_lo<H + 0, H + 0>(d, a0, b0, idesc_qk, 1u);
+          mma_ss_lo<H + 2, H + 2>(d, a0, b0, idesc_qk, 1u);
+          mma_ss_lo<H + 4, H + 4>(d, a0, b0, idesc_qk, 1u);
+          mma_ss_lo<H + 6, H + 6>(d, a0, b0, idesc_qk, 1u);
         }
       };
       auto issue_pv = [&](int t, int slot, bool acc) {
-#pragma unroll
-        for (int k = 0; k < kBlockN / 16; ++k) {
-          const uint64_t bd =
-              smem_desc_sw128(sKVa + slot * L::kTileBytes + k * 2048, L::kHalfBytes, 1024);
-          mma_bf16_ts(tmem + 256 + t * D, tmem + t * 128 + k * 8, bd, idesc_pv,
-                      (acc || k > 0) ? 1u : 0u);
-        }
+        const uint32_t b0 = desc_lo(sKVa + slot * L::kTileBytes, L::kHalfBytes);
+        const uint32_t d = tmem + 256 + t * D;
+        const uint32_t a = tmem + t * 128;
+        const uint32_t a1 = acc ? 1u : 0u;
+        mma_ts_lo<0 * 128>(d, a + 0, b0, idesc_pv, a1);
+        mma_ts_lo<1 * 128>(d, a + 8, b0, idesc_pv, 1u);
+        mma_ts_lo<2 * 128>(d, a + 16, b0, idesc_pv, 1u);
+        mma_ts_lo<3 * 128>(d, a + 24, b0, idesc_pv, 1u);
+        mma_ts_lo<4 * 128>(d, a + 32, b0, idesc_pv, 1u);
+        mma_ts_lo<5 * 128>(d, a + 40, b0, idesc_pv, 1u);
+        mma_ts_lo<6 * 128>(d, a + 48, b0, idesc_pv, 1u);
+        mma_ts_lo<7 * 128>(d, a + 56, b0, idesc_pv, 1u);
       };
       auto wait_kv = [&](int n) -> bool {
         if (!mbar_wait(&kv_full[n % NST], (n / NST) & 1, abort_flag, p.err)) return false;
         tc_fence_after();
         return true;
       };
-
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.err) && wait_kv(0);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        if (!(ok = mbar_wait(&unit_full[k & 1], (k >> 1) & 1, abort_flag, p.err))) break;
+        const int u = unit_ring[k & 1];
+        mbar_arrive(&unit_free[k & 1]);
+        if (u < 0) break;
+        const int c0 = k * tiles2;   // this unit's first K/V load
+        if (!(ok = mbar_wait(q_full, k & 1, abort_flag, p.err) && wait_kv(c0))) break;
+        issue_s(0, c0 % NST);
         mma_commit(&s_ready[0]);
-        issue_s(1, 0);
+        issue_s(1, c0 % NST);
         mma_commit(&s_ready[1]);
-        mma_commit(&kv_empty[0]);
-      }
-      for (int j = 0; ok && j < p.n_tiles; ++j) {
-        const int nv = 2 * j + 1, nk = 2 * j + 2;
-        const bool more = j + 1 < p.n_tiles;
-        if (!(ok = wait_kv(nv))) break;
-        if (!(ok = mbar_wait(&p_ready[0], j & 1, abort_flag, p.err))) break;
-        tc_fence_after();
-        issue_pv(0, nv % NST, j > 0);
-        if (more) {
-          if (!(ok = wait_kv(nk))) break;
-          issue_s(0, nk % NST);
-          mma_commit(&s_ready[0]);
-        } else {
-          mma_commit(&o_done[0]);
-        }
-        if (!(ok = mbar_wait(&p_ready[1], j & 1, abort_flag, p.err))) break;
-        tc_fence_after();
-        issue_pv(1, nv % NST, j > 0);
-        mma_commit(&kv_empty[nv % NST]);
-        if (more) {
-          issue_s(1, nk % NST);
-          mma_commit(&s_ready[1]);
-          mma_commit(&kv_empty[nk % NST]);
-        } else {
-          mma_commit(&o_done[1]);
+        mma_commit(&kv_empty[c0 % NST]);
+        if (p.n_tiles == 1) mma_commit(q_free);
+        for (int j = 0; ok && j < p.n_tiles; ++j) {
+          const int js = k * p.n_tiles + j;   // key-tile step over all units
+          const int nv = c0 + 2 * j + 1, nk = c0 + 2 * j + 2;
+          const bool more = j + 1 < p.n_tiles;
+          if (!(ok = wait_kv(nv))) break;
+          if (!(ok = mbar_wait(&p_ready[0], js & 1, abort_flag, p.err))) break;
+          // the previous unit's epilogue must have read O_0 before it is overwritten
+          if (j == 0 && k > 0 && !(ok = mbar_wait(&o_free[0], (k - 1) & 1, abort_flag, p.err)))
+            break;
+          tc_fence_after();
+          issue_pv(0, nv % NST, j > 0);
+          if (more) {
+            if (!(ok = wait_kv(nk))) break;
+            issue_s(0, nk % NST);
+            mma_commit(&s_ready[0]);
+          } else {
+            mma_commit(&o_done[0]);
+          }
+          if (!(ok = mbar_wait(&p_ready[1], js & 1, abort_flag, p.err))) break;
+          if (j == 0 && k > 0 && !(ok = mbar_wait(&o_free[1], (k - 1) & 1, abort_flag, p.err)))
+            break;
+          tc_fence_after();
+          issue_pv(1, nv % NST, j > 0);
+          mma_commit(&kv_empty[nv % NST]);
+          if (more) {
+            issue_s(1, nk % NST);
+            mma_commit(&s_ready[1]);
+            mma_commit(&kv_empty[nk % NST]);
+            if (j + 2 == p.n_tiles) mma_commit(q_free);   // the unit's last S MMAs
+          } else {
+            mma_commit(&o_done[1]);
+          }
         }
       }
       // Every MMA issued so far must finish before tensor memory is freed.
@@ -332,136 +455,141 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t tS = tmem + lane_base + t * 128;
     const uint32_t tO = tmem + lane_base + 256 + t * D;
     const float sl2 = p.scale_log2;
-
-    float m_run = -INFINITY;   // running max, log2 units (scaled)
-    float l_run = 0.f;         // running sum of 2^(s*sl2 - m_run)
+    uint8_t* stage = sStage + (warp - 4) * PS::kStageBytes;   // this warp's 32 x 128 B
     bool ok = true;
-    TileWalk w;
-    w.init(p);
-    for (int j = 0; j < p.n_tiles; ++j) {
-      if (!(ok = mbar_wait(&s_ready[t], j & 1, abort_flag, p.err))) break;
-      tc_fence_after();
-      // S in four 32-column chunks: chunk c + 1 is in flight while the row
-      // max of chunk c is taken (eight independent max chains)
-      float s[kBlockN];
-      float mx[8];
-      tmem_ld32(tS, s);
-      tmem_wait_ld_into(s);
-      tmem_ld32(tS + 32, s + 32);
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        mx[i] = max3f(s[4 * i], s[4 * i + 1], fmaxf(s[4 * i + 2], s[4 * i + 3]));
-#pragma unroll
-      for (int c = 1; c < kBlockN / 32; ++c) {
-        tmem_wait_ld_into(s + 32 * c);
-        if (c + 1 < kBlockN / 32) tmem_ld32(tS + 32 * (c + 1), s + 32 * (c + 1));
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          mx[i] = max3f(mx[i], s[32 * c + 4 * i], s[32 * c + 4 * i + 1]);
-          mx[i] = max3f(mx[i], s[32 * c + 4 * i + 2], s[32 * c + 4 * i + 3]);
+    for (int k = 0; ok; ++k) {
+      if (!(ok = mbar_wait(&unit_full[k & 1], (k >> 1) & 1, abort_flag, p.err))) break;
+      const int u = unit_ring[k & 1];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&unit_free[k & 1]);
+      if (u < 0) break;
+      float m_run = -INFINITY;   // running max, log2 units (scaled)
+      float l_run = 0.f;         // running sum of 2^(s*sl2 - m_run)
+      TileWalk w;
+      w.init(p);
+      for (int j = 0; j < p.n_tiles; ++j) {
+        const int js = k * p.n_tiles + j;   // key-tile step over all units
+        if (!(ok = mbar_wait(&s_ready[t], js & 1, abort_flag, p.err))) break;
+        if (p.merge && j == 0 && lane == 0) {
+          // the accumulator rows this warp merges into at the end of the unit
+          int b, h, q0;
+          decode(u, b, h, q0);
+          const int r0w = q0 + t * kBlockM + quarter * 32;
+          for (int c = 0; c < D / 32; ++c)
+            tma_prefetch_l2_5d(&p.tmap_out32, c * 32, r0w % p.seg_q, h, r0w / p.seg_q, b);
         }
-      }
-      const int valid = w.valid();
-      if (valid < kBlockN) {
-        // a chunk's last tile: columns past the chunk end are masked (rare,
-        // so the max is simply taken again over the masked row)
+        tc_fence_after();
+        // S in four 32-column chunks: chunk c + 1 is in flight while the row
+        // max of chunk c is taken (eight independent max chains)
+        float s[kBlockN];
+        float mx[8];
+        tmem_ld32(tS, s);
+        tmem_wait_ld_into(s);
+        tmem_ld32(tS + 32, s + 32);
 #pragma unroll
-        for (int c = 0; c < kBlockN; ++c)
-          if (c >= valid) s[c] = -INFINITY;
+        for (int i = 0; i < 8; ++i)
+          mx[i] = max3f(s[4 * i], s[4 * i + 1], fmaxf(s[4 * i + 2], s[4 * i + 3]));
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = s[i];
+        for (int c = 1; c < kBlockN / 32; ++c) {
+          tmem_wait_ld_into(s + 32 * c);
+          if (c + 1 < kBlockN / 32) tmem_ld32(tS + 32 * (c + 1), s + 32 * (c + 1));
 #pragma unroll
-        for (int c = 8; c < kBlockN; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
-      }
-      const float m_tile =
-          max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
-          sl2;
-      {
-        // Rescale the rows whose max moved beyond the threshold, then
-        // exponentiate on the MUFU unit, which maps the masked -inf columns
-        // of a tile cut by its chunk's end to exactly 0.
-        const bool need = m_tile > m_run + kRescaleThreshold;
-        if (__any_sync(0xffffffffu, need)) {
-          const float alpha = need ? ex2_approx(m_run - m_tile) : 1.0f;
-          if (need) {
-            l_run *= alpha;
-            m_run = m_tile;
+          for (int i = 0; i < 8; ++i) {
+            mx[i] = max3f(mx[i], s[32 * c + 4 * i], s[32 * c + 4 * i + 1]);
+            mx[i] = max3f(mx[i], s[32 * c + 4 * i + 2], s[32 * c + 4 * i + 3]);
           }
-          if (j > 0) {
+        }
+        const int valid = w.valid();
+        if (valid < kBlockN) {
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              float o[32];
-              tmem_ld32(tO + c * 32, o);
-              tmem_wait_ld_into(o);
+          for (int c = 0; c < kBlockN; ++c)
+            if (c >= valid) s[c] = -INFINITY;
 #pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] *= alpha;
-              tmem_st32(tO + c * 32, o);
+          for (int i = 0; i < 8; ++i) mx[i] = s[i];
+#pragma unroll
+          for (int c = 8; c < kBlockN; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
+        }
+        const float m_tile =
+            max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
+            sl2;
+        {
+          const bool need = m_tile > m_run + kRescaleThreshold;
+          if (__any_sync(0xffffffffu, need)) {
+            const float alpha = need ? ex2_approx(m_run - m_tile) : 1.0f;
+            if (need) {
+              l_run *= alpha;
+              m_run = m_tile;
+            }
+            if (j > 0) {
+#pragma unroll
+              for (int c = 0; c < D / 32; ++c) {
+                float o[32];
+                tmem_ld32(tO + c * 32, o);
+                tmem_wait_ld_into(o);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) o[i] *= alpha;
+                tmem_st32(tO + c * 32, o);
+              }
             }
           }
-        }
-        const float2 sl2x2 = make_float2(sl2, sl2), nmx2 = make_float2(-m_run, -m_run);
-        float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+          const float2 sl2x2 = make_float2(sl2, sl2), nmx2 = make_float2(-m_run, -m_run);
+          float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
-        for (int c = 0; c < kBlockN / 32; ++c) {
-          uint32_t pk[16];
+          for (int c = 0; c < kBlockN / 32; ++c) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int e = c * 32 + 2 * i;
-            const float2 x = fma2(make_float2(s[e], s[e + 1]), sl2x2, nmx2);
-            const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            acc[i & 3] = add2(acc[i & 3], pp);
-            pk[i] = pack_bf16x2(pp.x, pp.y);
+            for (int i = 0; i < 16; ++i) {
+              const int e = c * 32 + 2 * i;
+              const float2 x = fma2(make_float2(s[e], s[e + 1]), sl2x2, nmx2);
+              const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+              acc[i & 3] = add2(acc[i & 3], pp);
+              pk[i] = pack_bf16x2(pp.x, pp.y);
+            }
+            tmem_st16(tS + c * 16, pk);
           }
-          tmem_st16(tS + c * 16, pk);
+          const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
+          l_run += (a01.x + a01.y) + (a23.x + a23.y);
         }
-        const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
-        l_run += (a01.x + a01.y) + (a23.x + a23.y);
-      }
-      if (t == 0 && valid < kBlockN) {
-        // Ring Anything trim, V side: a chunk's last tile was loaded whole,
-        // and the rows past the chunk end may be padding of any value (a
-        // padded all-gather slot).  Their P is exactly 0, but 0 * NaN is
-        // NaN in the MMA, so the rows are zeroed in shared memory before
-        // P V reads them.  Tile 0's P V is issued first and the slot is not
-        // refilled before both tiles have consumed it.
-        const int n = 2 * j + 1;
-        if (!(ok = mbar_wait(&kv_full[n % NST], (n / NST) & 1, abort_flag, p.err))) break;
-        if (row >= valid) {
-          uint8_t* vrow = sKV + (n % NST) * L::kTileBytes + row * 128;
+        if (t == 0 && valid < kBlockN) {
+          const int n = k * tiles2 + 2 * j + 1;
+          if (!(ok = mbar_wait(&kv_full[n % NST], (n / NST) & 1, abort_flag, p.err))) break;
+          if (row >= valid) {
+            uint8_t* vrow = sKV + (n % NST) * L::kTileBytes + row * 128;
 #pragma unroll
-          for (int hh = 0; hh < D / 64; ++hh)
+            for (int hh = 0; hh < D / 64; ++hh)
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              reinterpret_cast<uint4*>(vrow + hh * L::kHalfBytes)[k] = make_uint4(0, 0, 0, 0);
+              for (int kk = 0; kk < 8; ++kk)
+                reinterpret_cast<uint4*>(vrow + hh * L::kHalfBytes)[kk] = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_ready[t]);
+        w.next(p);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_ready[t]);
-      w.next(p);
-    }
-    int rounds = 0;   // epilogue rounds staged (phase of epi_full / epi_free)
-    if (ok && mbar_wait(&o_done[t], 0, abort_flag, p.err)) {
+      if (!ok) break;
+      int b, h, q0;
+      decode(u, b, h, q0);
+      const int r0w = q0 + t * kBlockM + quarter * 32;     // first row of this warp
+      if (!(ok = mbar_wait(&o_done[t], k & 1, abort_flag, p.err))) break;
       tc_fence_after();
-      // Epilogue: O / l goes through this tile's Q buffer (idle once o_done
-      // fired) in 128-byte swizzled boxes of 128 rows, and leaves with TMA
-      // stores; rows past S_q are clipped by the tensor map.  The warps hand
-      // the staging buffer to the storing thread and back through bounded
-      // mbarrier waits, so a warp that gave up never blocks the others.
+      // ---- epilogue, per warp (its 32 rows), in rounds of 128 bytes of
+      // columns: O from tensor memory, scaled (and merged) into the warp's
+      // 4 KB staging area in the 128-byte swizzled layout, stored with one
+      // 32-row TMA box.  The staging area is reused once the previous
+      // round's store has read it.
       const int s_row = q0 + t * kBlockM + row;
       const float lse_c = (m_run + log2f(l_run)) * 0.69314718055994530942f;
-      float o_w = 1.0f / l_run;   // weight of the raw accumulator O
-      float acc_w = 0.f;          // merge mode: weight of the (out, lse) already there
+      float o_w = 1.0f / l_run;
+      float acc_w = 0.f;
       const long long l_off = b * p.l_sb + h * p.l_sh + (long long)s_row * p.l_ss;
       float* lse_p = p.lse != nullptr && s_row < p.S_q &&
                              CP_IN_BOUNDS(l_off >= 0 && l_off < p.span_lse, p.err)
                          ? p.lse + l_off
                          : nullptr;
       if (p.merge) {
-        // fp32 log-sum-exp merge with the accumulator (ContextParallelConfig
-        // .convert_to_fp32): lse' = max + log1p(exp(-|a - b|))
         const float a = lse_p ? *lse_p : -INFINITY;
         const float mx = fmaxf(a, lse_c);
         const float nl = a == -INFINITY ? lse_c : mx + log1pf(expf(-fabsf(a - lse_c)));
@@ -471,88 +599,104 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       } else if (lse_p) {
         *lse_p = lse_c;
       }
-      const float inv_l = o_w;
-      uint8_t* stage = sQ + t * L::kTileBytes;
-      const int esz = p.out_bf16 ? 2 : 4;
-      const int cols_per_box = 128 / esz;               // 32 fp32 or 64 bf16
-      const int boxes = D / cols_per_box;               // per 128-row tile
-      const int boxes_per_round = L::kTileBytes / (128 * 128);
-      const bool leader = (warp & 3) == 0 && lane == 0;
-      for (int b0 = 0; ok && b0 < boxes; b0 += boxes_per_round, ++rounds) {
-        // the previous round's TMA stores must have read the staging buffer
-        if (rounds > 0 && !(ok = mbar_wait(&epi_free[t], (rounds - 1) & 1, abort_flag, p.err)))
-          break;
-        const int r0 = q0 + t * kBlockM;
-        if (p.merge) {
-          // bring this round's accumulator boxes into the staging buffer
-          if (leader) {
-            mbar_arrive_expect_tx(&acc_full[t], boxes_per_round * (128 * 128));
-            for (int bx = b0; bx < b0 + boxes_per_round; ++bx)
-              tma_load_5d(stage + (bx - b0) * (128 * 128), &p.tmap_out, &acc_full[t],
-                          bx * cols_per_box, r0 % p.seg_q, h, r0 / p.seg_q, b);
-          }
-          if (!(ok = mbar_wait(&acc_full[t], rounds & 1, abort_flag, p.err))) break;
-        }
-        for (int bx = b0; bx < b0 + boxes_per_round; ++bx) {
-          uint8_t* box = stage + (bx - b0) * (128 * 128) + row * 128;
-          // this box holds O columns [bx * cols_per_box, (bx+1) * cols_per_box)
-          if (p.merge) {          // fp32 accumulator: out' = acc_w * out + o_w * O
-            float o[32];
-            tmem_ld32(tO + bx * 32, o);
-            tmem_wait_ld_into(o);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              float4* cell = reinterpret_cast<float4*>(box + ((k ^ (row & 7)) << 4));
-              const float4 a4 = *cell;
-              *cell = make_float4(fmaf(acc_w, a4.x, o[4 * k] * inv_l),
-                                  fmaf(acc_w, a4.y, o[4 * k + 1] * inv_l),
-                                  fmaf(acc_w, a4.z, o[4 * k + 2] * inv_l),
-                                  fmaf(acc_w, a4.w, o[4 * k + 3] * inv_l));
-            }
-          } else if (p.out_bf16) {
-#pragma unroll
-            for (int hlf = 0; hlf < 2; ++hlf) {
-              float o[32];
-              tmem_ld32(tO + bx * 64 + hlf * 32, o);
-              tmem_wait_ld_into(o);
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                uint4 v;
-                v.x = pack_bf16x2(o[8 * k + 0] * inv_l, o[8 * k + 1] * inv_l);
-                v.y = pack_bf16x2(o[8 * k + 2] * inv_l, o[8 * k + 3] * inv_l);
-                v.z = pack_bf16x2(o[8 * k + 4] * inv_l, o[8 * k + 5] * inv_l);
-                v.w = pack_bf16x2(o[8 * k + 6] * inv_l, o[8 * k + 7] * inv_l);
-                const int chunk = hlf * 4 + k;
-                *reinterpret_cast<uint4*>(box + ((chunk ^ (row & 7)) << 4)) = v;
-              }
-            }
-          } else {
-            float o[32];
-            tmem_ld32(tO + bx * 32, o);
-            tmem_wait_ld_into(o);
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              *reinterpret_cast<float4*>(box + ((k ^ (row & 7)) << 4)) =
-                  make_float4(o[4 * k] * inv_l, o[4 * k + 1] * inv_l, o[4 * k + 2] * inv_l,
-                              o[4 * k + 3] * inv_l);
-          }
-        }
+      const int c1 = r0w % p.seg_q, c3 = r0w / p.seg_q;    // its TMA row / segment coordinates
+      uint8_t* cell_row = stage + lane * 128;
+      // the previous round's store must have read the staging area before it
+      // is written again (the wait overlaps this round's TMEM load and math)
+      auto staging_free = [&]() {
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+      };
+      auto store_box = [&](int col0) {
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&epi_full[t]);
-        if (leader) {
-          if (!(ok = mbar_wait(&epi_full[t], rounds & 1, abort_flag, p.err))) break;
-          for (int bx = b0; bx < b0 + boxes_per_round; ++bx)
-            tma_store_5d(&p.tmap_out, stage + (bx - b0) * (128 * 128), bx * cols_per_box,
-                         r0 % p.seg_q, h, r0 / p.seg_q, b);
+        if (lane == 0) {
+          tma_store_5d(&p.tmap_out32, stage, col0, c1, h, c3, b);
           bulk_commit();
-          bulk_wait_read_all();
-          mbar_arrive(&epi_free[t]);
+        }
+      };
+      if (p.merge) {
+        // per round: the accumulator box (already pulled into L2 when the
+        // unit started) into the staging area, merged with O in place, stored
+        uint64_t* abar = &acc_bar[warp - 4];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          staging_free();
+          if (lane == 0) {
+            mbar_arrive_expect_tx(abar, 32 * 128);
+            tma_load_5d(stage, &p.tmap_out32, abar, c * 32, c1, h, c3, b);
+          }
+          float o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld_into(o);
+          if (c == D / 32 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&o_free[t]);
+          }
+          if (!(ok = mbar_wait(abar, (k * (D / 32) + c) & 1, abort_flag, p.err))) break;
+#pragma unroll
+          for (int kq = 0; kq < 8; ++kq) {
+            float4* cell = reinterpret_cast<float4*>(cell_row + ((kq ^ (lane & 7)) << 4));
+            const float4 a4 = *cell;
+            *cell = make_float4(fmaf(acc_w, a4.x, o[4 * kq] * o_w),
+                                fmaf(acc_w, a4.y, o[4 * kq + 1] * o_w),
+                                fmaf(acc_w, a4.z, o[4 * kq + 2] * o_w),
+                                fmaf(acc_w, a4.w, o[4 * kq + 3] * o_w));
+          }
+          store_box(c * 32);
+        }
+        if (!ok) break;
+      } else if (p.out_bf16) {
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+#pragma unroll
+          for (int hlf = 0; hlf < 2; ++hlf) {
+            float o[32];
+            tmem_ld32(tO + c * 64 + hlf * 32, o);
+            tmem_wait_ld_into(o);
+            if (c == D / 64 - 1 && hlf == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&o_free[t]);
+            }
+            if (hlf == 0) staging_free();
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq) {
+              uint4 v;
+              v.x = pack_bf16x2(o[8 * kq + 0] * o_w, o[8 * kq + 1] * o_w);
+              v.y = pack_bf16x2(o[8 * kq + 2] * o_w, o[8 * kq + 3] * o_w);
+              v.z = pack_bf16x2(o[8 * kq + 4] * o_w, o[8 * kq + 5] * o_w);
+              v.w = pack_bf16x2(o[8 * kq + 6] * o_w, o[8 * kq + 7] * o_w);
+              const int chunk = hlf * 4 + kq;
+              *reinterpret_cast<uint4*>(cell_row + ((chunk ^ (lane & 7)) << 4)) = v;
+            }
+          }
+          store_box(c * 64);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld_into(o);
+          if (c == D / 32 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&o_free[t]);
+          }
+          staging_free();
+#pragma unroll
+          for (int kq = 0; kq < 8; ++kq)
+            *reinterpret_cast<float4*>(cell_row + ((kq ^ (lane & 7)) << 4)) =
+                make_float4(o[4 * kq] * o_w, o[4 * kq + 1] * o_w, o[4 * kq + 2] * o_w,
+                            o[4 * kq + 3] * o_w);
+          store_box(c * 32);
         }
       }
     }
     // shared memory must not be released while TMA still reads it
-    if (rounds > 0) mbar_wait_drain(&epi_free[t], (rounds - 1) & 1, p.err);
+    if (lane == 0) bulk_wait_read_all();
   }
 
   tc_fence_before();
@@ -564,7 +708,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 // ------------------------------------------------------------------ host side
+// Work counters of the persistent grid: kUnitSlots pairs per device (next
+// unit, CTAs done), zero between launches.  Launches take the pairs in turn,
+// so launches in flight at the same time on different streams use different
+// pairs unless more than kUnitSlots of them overlap.
+constexpr int kUnitSlots = 64;
+__device__ unsigned int g_unit_counters[2 * kUnitSlots];
+
 namespace {
+
+unsigned int* unit_counters(int dev) {
+  static std::atomic<unsigned int*> addr[64];
+  unsigned int* a = addr[dev].load(std::memory_order_acquire);
+  if (!a) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_unit_counters) != cudaSuccess) return nullptr;
+    a = static_cast<unsigned int*>(p);
+    addr[dev].store(a, std::memory_order_release);
+  }
+  return a;
+}
+
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -614,13 +778,13 @@ int encode_in(CUtensorMap* map, const TensorView& t) {
 }
 
 // Output (f32 or bf16) -> 5-D map with 128-byte, 128-row boxes.
-int encode_out(CUtensorMap* map, const TensorView& t) {
+int encode_out(CUtensorMap* map, const TensorView& t, int box_rows = 128) {
   auto fn = get_encode_fn();
   if (!fn) return CP_ERR_CUDA;
   const int es = dtype_size(t.dtype);
   cuuint64_t dims[5], strides[4];
   seg_geometry(t, dims, strides);
-  const cuuint32_t box[5] = {(cuuint32_t)(128 / es), 128, 1, 1, 1};
+  const cuuint32_t box[5] = {(cuuint32_t)(128 / es), (cuuint32_t)box_rows, 1, 1, 1};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = fn(map, t.dtype == CP_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
@@ -632,7 +796,7 @@ int encode_out(CUtensorMap* map, const TensorView& t) {
 
 template <int D, int NST>
 int launch_tc(const AttnTcParams& prm, int grid, cudaStream_t stream) {
-  constexpr size_t smem = 1024 + (2 + NST) * (size_t)TcSmem<D>::kTileBytes + 256;
+  constexpr size_t smem = PersistSmem<D, NST>::kBytes;
   auto kern = attn_ring_tc_kernel<D, NST>;
   static bool configured[64] = {};
   int dev = 0;
@@ -670,6 +834,7 @@ int launch_attn_ring_tc(const RingArgs& a, cudaStream_t stream) {
   if ((st = encode_in(&prm.tmap_k, a.k)) != CP_OK) return st;
   if ((st = encode_in(&prm.tmap_v, a.v)) != CP_OK) return st;
   if ((st = encode_out(&prm.tmap_out, a.out)) != CP_OK) return st;
+  if ((st = encode_out(&prm.tmap_out32, a.out, 32)) != CP_OK) return st;
   prm.out = a.out.data;
   prm.out_bf16 = a.out.dtype == CP_BF16;
   prm.merge = a.merge ? 1 : 0;
@@ -681,6 +846,18 @@ int launch_attn_ring_tc(const RingArgs& a, cudaStream_t stream) {
   prm.G_q = a.q.ndim == 5 ? (int)a.q.shape[0] : 1;
   prm.G_kv = a.k.ndim == 5 ? (int)a.k.shape[0] : 1;
   prm.span_lse = span_elems(a.lse);
+  prm.span_out = span_elems(a.out);
+  if (a.out.ndim == 5) {
+    prm.o_sg = a.out.stride[0];
+    prm.o_sb = a.out.stride[1];
+    prm.o_ss = a.out.stride[2];
+    prm.o_sh = a.out.stride[3];
+  } else {
+    prm.o_sg = 0;
+    prm.o_sb = a.out.stride[0];
+    prm.o_ss = a.out.stride[1];
+    prm.o_sh = a.out.stride[2];
+  }
   if (a.q.ndim == 5) {   // [G, B, S/G, H, D] shards, read in place
     prm.B = (int)a.q.shape[1];
     prm.seg_q = (int)a.q.shape[2];
@@ -710,9 +887,24 @@ int launch_attn_ring_tc(const RingArgs& a, cudaStream_t stream) {
   }
   prm.n_tiles = n_tiles;
   prm.scale_log2 = a.scale * 1.4426950408889634f;
-  const long long grid = (long long)prm.n_q_blocks * prm.H * prm.B;
-  if (grid <= 0 || n_tiles <= 0) return CP_OK;
-  if (grid > 0x7fffffffLL) return CP_ERR_SHAPE;
+  const long long units = (long long)prm.n_q_blocks * prm.H * prm.B;
+  if (units <= 0 || n_tiles <= 0) return CP_OK;
+  if (units > 0x7fffffffLL) return CP_ERR_SHAPE;
+  prm.n_units = (int)units;
+  // persistent: one CTA per SM walks the units round-robin
+  static int sm_count[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CP_ERR_CUDA;
+  if (sm_count[dev] == 0 &&
+      cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return CP_ERR_CUDA;
+  const long long grid = units < sm_count[dev] ? units : sm_count[dev];
+  // a counter pair for this launch, round-robin over kUnitSlots pairs; each
+  // launch's last CTA leaves its pair at zero
+  unsigned int* ctr = unit_counters(dev);
+  if (!ctr) return CP_ERR_CUDA;
+  static std::atomic<unsigned> seq[64];
+  prm.unit_ctr = ctr + 2 * (seq[dev].fetch_add(1, std::memory_order_relaxed) % kUnitSlots);
   const int D = (int)a.q.shape[a.q.ndim - 1];
   if (D == 128) return launch_tc<128, kStagesD128>(prm, (int)grid, stream);
   if (D == 64) return launch_tc<64, kStagesD64>(prm, (int)grid, stream);

@@ -42,6 +42,11 @@
  *    CP_BF16; lse always CP_F32.  TMA needs 16-byte-aligned base pointers and
  *    strides for bf16 inputs.
  *  - Empty key sets give out = 0 and lse = -inf (the merge identity).
+ *  - The bf16 attention runs on a persistent grid (one CTA per SM) that takes
+ *    its work units from a device counter pair owned by the library; each
+ *    launch takes the next of 64 pairs per device and leaves it at zero.  So
+ *    at most 64 of these launches may execute at the same time on one device
+ *    (from different streams); more could share a pair and skip work.
  */
 #ifndef CPATTN_H_
 #define CPATTN_H_
