@@ -21,12 +21,17 @@
 //   warp 0      TMA producer: per unit Q (once the previous unit's last S
 //               MMAs have read the Q buffer), then K_j, V_j into a ring of
 //               NST slots
-//   warp 1      MMA issuer (one thread): S_t = Q_t K^T, O_t += P_t V; the
+//   warp 1      MMA issuer (lane 0): S_t = Q_t K^T, O_t += P_t V; the
 //               first P V of a unit waits until the previous unit's epilogue
 //               has read O_t out of tensor memory
-//   warp 2      tensor-memory allocator
+//   warp 2      tensor-memory allocator, then the watchdog of the P barriers
 //   warps 4-7   softmax + epilogue of query tile 0 (one row per thread)
 //   warps 8-11  softmax + epilogue of query tile 1
+// The softmax warps publish P_t on a hardware named barrier (arrive) that
+// the MMA warp syncs on.  A shared-memory signal (an mbarrier or a flag)
+// would be observed late: the MMA warp's polls queue behind the softmax
+// warps' MUFU instructions on the same sub-partition (~150-250 clocks per
+// poll, measured).  Every other hand-off uses mbarriers with bounded waits.
 // Epilogue, per warp and its 32 rows: O in rounds of 128 bytes of columns
 // from tensor memory, scaled (or, for the fp32 accumulator, merged with the
 // box the same warp TMA-loads), staged in the warp's own 4 KB of shared
@@ -84,6 +89,10 @@ constexpr int kStagesD64 = 6;                    // 32 KB Q + NST x 16 KB
 // at this split neither role spills.
 constexpr int kRegsControl = 72;
 constexpr int kRegsSoftmax = 216;
+// Named barriers on which P_t is published: id 1 + t, the four softmax warps
+// of query tile t (arrive) and the MMA warp (sync).
+constexpr uint32_t kPBarBase = 1;
+constexpr uint32_t kPBarThreads = (kBlockM / 32 + 1) * 32;
 
 struct AttnTcParams {
   // 5-D maps {D, seg, H, G, B}: token s of the sequence is row s % seg of
@@ -218,8 +227,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* kv_full = bars + 2;
   uint64_t* kv_empty = kv_full + NST;
   uint64_t* s_ready = kv_empty + NST;   // [2]
-  uint64_t* p_ready = s_ready + 2;      // [2]
-  uint64_t* o_done = p_ready + 2;       // [2]
+  uint64_t* o_done = s_ready + 2;       // [2]
   uint64_t* o_free = o_done + 2;        // [2] the epilogue has read O_t out of tensor memory
   uint64_t* drain = o_free + 2;         // [1]
   uint64_t* acc_bar = drain + 1;        // [8] merge mode: a warp's accumulator box is in staging
@@ -229,6 +237,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   volatile int* unit_ring = unit_ring_raw;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unit_ring_raw + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* mma_exited = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -242,7 +251,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_ready[t], 1);
-      mbar_init(&p_ready[t], kBlockM / 32);   // one arrive per softmax warp
       mbar_init(&o_done[t], 1);
       mbar_init(&o_free[t], kBlockM / 32);    // one arrive per softmax warp
     }
@@ -253,6 +261,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int i = 0; i < 8; ++i) mbar_init(&acc_bar[i], 1);
     *abort_flag = 0;
+    *mma_exited = 0;
     fence_barrier_init();
   }
   if (warp == 2) {
@@ -350,99 +359,152 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, D, true);
-      const uint32_t sQa = smem_u32(sQ);
-      const uint32_t sKVa = smem_u32(sKV);
-      // descriptor low words: start address (16-byte units) | LBO << 16; the
-      // k-steps of one MMA group add compile-time offsets to one base
-      auto issue_s = [&](int t, int slot) {
-        const uint32_t a0 = desc_lo(sQa + t * L::kTileBytes, 16);
-        const uint32_t b0 = desc_lo(sKVa + slot * L::kTileBytes, 16);
-        const uint32_t d = tmem + t * 128;
-        mma_ss_lo<0, 0>(d, a0, b0, idesc_qk, 0u);
-        mma_ss_lo<2, 2>(d, a0, b0, idesc_qk, 1u);
-        mma_ss_lo<4, 4>(d, a0, b0, idesc_qk, 1u);
-        mma_ss_lo<6, 6>(d, a0, b0, idesc_qk, 1u);
-        if constexpr (D == 128) {
-          constexpr uint32_t H = L::kHalfBytes >> 4;
-          mma_ss_lo<H + 0, H + 0>(d, a0, b0, idesc_qk, 1u);
-          mma_ss_lo<H + 2, H + 2>(d, a0, b0, idesc_qk, 1u);
-          mma_ss_lo<H + 4, H + 4>(d, a0, b0, idesc_qk, 1u);
-          mma_ss_lo<H + 6, H + 6>(d, a0, b0, idesc_qk, 1u);
-        }
-      };
-      auto issue_pv = [&](int t, int slot, bool acc) {
-        const uint32_t b0 = desc_lo(sKVa + slot * L::kTileBytes, L::kHalfBytes);
-        const uint32_t d = tmem + 256 + t * D;
-        const uint32_t a = tmem + t * 128;
-        const uint32_t a1 = acc ? 1u : 0u;
-        mma_ts_lo<0 * 128>(d, a + 0, b0, idesc_pv, a1);
-        mma_ts_lo<1 * 128>(d, a + 8, b0, idesc_pv, 1u);
-        mma_ts_lo<2 * 128>(d, a + 16, b0, idesc_pv, 1u);
-        mma_ts_lo<3 * 128>(d, a + 24, b0, idesc_pv, 1u);
-        mma_ts_lo<4 * 128>(d, a + 32, b0, idesc_pv, 1u);
-        mma_ts_lo<5 * 128>(d, a + 40, b0, idesc_pv, 1u);
-        mma_ts_lo<6 * 128>(d, a + 48, b0, idesc_pv, 1u);
-        mma_ts_lo<7 * 128>(d, a + 56, b0, idesc_pv, 1u);
-      };
-      auto wait_kv = [&](int n) -> bool {
-        if (!mbar_wait(&kv_full[n % NST], (n / NST) & 1, abort_flag, p.err)) return false;
-        tc_fence_after();
-        return true;
-      };
-      bool ok = true;
-      for (int k = 0; ok; ++k) {
-        if (!(ok = mbar_wait(&unit_full[k & 1], (k >> 1) & 1, abort_flag, p.err))) break;
-        const int u = unit_ring[k & 1];
-        mbar_arrive(&unit_free[k & 1]);
-        if (u < 0) break;
-        const int c0 = k * tiles2;   // this unit's first K/V load
-        if (!(ok = mbar_wait(q_full, k & 1, abort_flag, p.err) && wait_kv(c0))) break;
-        issue_s(0, c0 % NST);
-        mma_commit(&s_ready[0]);
-        issue_s(1, c0 % NST);
-        mma_commit(&s_ready[1]);
-        mma_commit(&kv_empty[c0 % NST]);
-        if (p.n_tiles == 1) mma_commit(q_free);
-        for (int j = 0; ok && j < p.n_tiles; ++j) {
-          const int js = k * p.n_tiles + j;   // key-tile step over all units
-          const int nv = c0 + 2 * j + 1, nk = c0 + 2 * j + 2;
-          const bool more = j + 1 < p.n_tiles;
-          if (!(ok = wait_kv(nv))) break;
-          if (!(ok = mbar_wait(&p_ready[0], js & 1, abort_flag, p.err))) break;
-          // the previous unit's epilogue must have read O_0 before it is overwritten
-          if (j == 0 && k > 0 && !(ok = mbar_wait(&o_free[0], (k - 1) & 1, abort_flag, p.err)))
-            break;
-          tc_fence_after();
-          issue_pv(0, nv % NST, j > 0);
-          if (more) {
-            if (!(ok = wait_kv(nk))) break;
-            issue_s(0, nk % NST);
-            mma_commit(&s_ready[0]);
-          } else {
-            mma_commit(&o_done[0]);
-          }
-          if (!(ok = mbar_wait(&p_ready[1], js & 1, abort_flag, p.err))) break;
-          if (j == 0 && k > 0 && !(ok = mbar_wait(&o_free[1], (k - 1) & 1, abort_flag, p.err)))
-            break;
-          tc_fence_after();
-          issue_pv(1, nv % NST, j > 0);
-          mma_commit(&kv_empty[nv % NST]);
-          if (more) {
-            issue_s(1, nk % NST);
-            mma_commit(&s_ready[1]);
-            mma_commit(&kv_empty[nk % NST]);
-            if (j + 2 == p.n_tiles) mma_commit(q_free);   // the unit's last S MMAs
-          } else {
-            mma_commit(&o_done[1]);
-          }
+    // Lane 0 waits on the mbarriers and issues; the whole warp takes part in
+    // the named barriers on which P is published, so every branch below is
+    // taken by the whole warp with lane 0's outcome.
+    constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, false);
+    constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, D, true);
+    const uint32_t sQa = smem_u32(sQ);
+    const uint32_t sKVa = smem_u32(sKV);
+    // descriptor low words: start address (16-byte units) | LBO << 16; the
+    // k-steps of one MMA group add compile-time offsets to one base
+    auto issue_s = [&](int t, int slot) {
+      const uint32_t a0 = desc_lo(sQa + t * L::kTileBytes, 16);
+      const uint32_t b0 = desc_lo(sKVa + slot * L::kTileBytes, 16);
+      const uint32_t d = tmem + t * 128;
+      mma_ss_lo<0, 0>(d, a0, b0, idesc_qk, 0u);
+      mma_ss_lo<2, 2>(d, a0, b0, idesc_qk, 1u);
+      mma_ss_lo<4, 4>(d, a0, b0, idesc_qk, 1u);
+      mma_ss_lo<6, 6>(d, a0, b0, idesc_qk, 1u);
+      if constexpr (D == 128) {
+        constexpr uint32_t H = L::kHalfBytes >> 4;
+        mma_ss_lo<H + 0, H + 0>(d, a0, b0, idesc_qk, 1u);
+        mma_ss_lo<H + 2, H + 2>(d, a0, b0, idesc_qk, 1u);
+        mma_ss_lo<H + 4, H + 4>(d, a0, b0, idesc_qk, 1u);
+        mma_ss_lo<H + 6, H + 6>(d, a0, b0, idesc_qk, 1u);
+      }
+    };
+    auto issue_pv = [&](int t, int slot, bool acc) {
+      const uint32_t b0 = desc_lo(sKVa + slot * L::kTileBytes, L::kHalfBytes);
+      const uint32_t d = tmem + 256 + t * D;
+      const uint32_t a = tmem + t * 128;
+      const uint32_t a1 = acc ? 1u : 0u;
+      mma_ts_lo<0 * 128>(d, a + 0, b0, idesc_pv, a1);
+      mma_ts_lo<1 * 128>(d, a + 8, b0, idesc_pv, 1u);
+      mma_ts_lo<2 * 128>(d, a + 16, b0, idesc_pv, 1u);
+      mma_ts_lo<3 * 128>(d, a + 24, b0, idesc_pv, 1u);
+      mma_ts_lo<4 * 128>(d, a + 32, b0, idesc_pv, 1u);
+      mma_ts_lo<5 * 128>(d, a + 40, b0, idesc_pv, 1u);
+      mma_ts_lo<6 * 128>(d, a + 48, b0, idesc_pv, 1u);
+      mma_ts_lo<7 * 128>(d, a + 56, b0, idesc_pv, 1u);
+    };
+    auto wait_kv = [&](int n) -> bool {
+      if (!mbar_wait(&kv_full[n % NST], (n / NST) & 1, abort_flag, p.err)) return false;
+      tc_fence_after();
+      return true;
+    };
+    auto warp_ok = [&](bool v) { return __shfl_sync(0xffffffffu, v ? 1 : 0, 0) != 0; };
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      int u = -1;
+      if (lane == 0) {
+        ok = mbar_wait(&unit_full[k & 1], (k >> 1) & 1, abort_flag, p.err);
+        if (ok) {
+          u = unit_ring[k & 1];
+          mbar_arrive(&unit_free[k & 1]);
         }
       }
+      ok = warp_ok(ok);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (!ok || u < 0) break;
+      const int c0 = k * tiles2;   // this unit's first K/V load
+      if (lane == 0) {
+        ok = mbar_wait(q_full, k & 1, abort_flag, p.err) && wait_kv(c0);
+        if (ok) {
+          issue_s(0, c0 % NST);
+          mma_commit(&s_ready[0]);
+          issue_s(1, c0 % NST);
+          mma_commit(&s_ready[1]);
+          mma_commit(&kv_empty[c0 % NST]);
+          if (p.n_tiles == 1) mma_commit(q_free);
+        }
+      }
+      ok = warp_ok(ok);
+      for (int j = 0; ok && j < p.n_tiles; ++j) {
+        const int nv = c0 + 2 * j + 1, nk = c0 + 2 * j + 2;
+        const bool more = j + 1 < p.n_tiles;
+        if (lane == 0) ok = wait_kv(nv);
+        if (!(ok = warp_ok(ok))) break;
+        named_sync(kPBarBase + 0, kPBarThreads);   // the tile-0 softmax warps published P_0
+        if (lane == 0) {
+          // the previous unit's epilogue must have read O_0 before it is overwritten
+          if (j == 0 && k > 0) ok = mbar_wait(&o_free[0], (k - 1) & 1, abort_flag, p.err);
+          if (ok) {
+            tc_fence_after();
+            issue_pv(0, nv % NST, j > 0);
+            if (more) {
+              ok = wait_kv(nk);
+              if (ok) {
+                issue_s(0, nk % NST);
+                mma_commit(&s_ready[0]);
+              }
+            } else {
+              mma_commit(&o_done[0]);
+            }
+          }
+        }
+        if (!(ok = warp_ok(ok))) break;
+        named_sync(kPBarBase + 1, kPBarThreads);   // P_1 published
+        if (lane == 0) {
+          if (j == 0 && k > 0) ok = mbar_wait(&o_free[1], (k - 1) & 1, abort_flag, p.err);
+          if (ok) {
+            tc_fence_after();
+            issue_pv(1, nv % NST, j > 0);
+            mma_commit(&kv_empty[nv % NST]);
+            if (more) {
+              issue_s(1, nk % NST);
+              mma_commit(&s_ready[1]);
+              mma_commit(&kv_empty[nk % NST]);
+              if (j + 2 == p.n_tiles) mma_commit(q_free);   // the unit's last S MMAs
+            } else {
+              mma_commit(&o_done[1]);
+            }
+          }
+        }
+        ok = warp_ok(ok);
+      }
+    }
+    if (lane == 0) {
+      *mma_exited = 1;
       // Every MMA issued so far must finish before tensor memory is freed.
       mma_commit(drain);
       mbar_wait_drain(drain, 0, p.err);
+    }
+    __syncwarp();
+   } else if (warp == 2) {
+    // ------------------------------------------------------------ watchdog
+    // The MMA warp's named-barrier syncs have no time limit.  A softmax warp
+    // stops arriving only after a bounded wait has failed, which raises the
+    // abort flag first; from then on this warp arrives on both P barriers
+    // every microsecond, releasing any sync the softmax warps no longer
+    // serve, until the MMA warp has left its loop (all its other waits are
+    // bounded and return at once once the flag is up).
+    const uint64_t t0 = globaltimer_ns();
+    uint64_t t_abort = 0;
+    for (;;) {
+      int state = 0;
+      if (lane == 0) state = (*mma_exited ? 1 : 0) | (*abort_flag ? 2 : 0);
+      state = __shfl_sync(0xffffffffu, state, 0);
+      if (state & 1) break;
+      const uint64_t now = globaltimer_ns();
+      if (state & 2) {
+        if (t_abort == 0) t_abort = now;
+        named_arrive(kPBarBase + 0, kPBarThreads);
+        named_arrive(kPBarBase + 1, kPBarThreads);
+        if (now - t_abort > 4 * kWaitTimeoutNs) break;
+      }
+      if (now - t0 > 64 * kWaitTimeoutNs) break;
+      __nanosleep(1000);
     }
    }
   } else {
@@ -479,26 +541,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tma_prefetch_l2_5d(&p.tmap_out32, c * 32, r0w % p.seg_q, h, r0w / p.seg_q, b);
         }
         tc_fence_after();
-        // S in four 32-column chunks: chunk c + 1 is in flight while the row
-        // max of chunk c is taken (eight independent max chains)
+        // S in one round trip: four 32-column loads behind one wait (the
+        // load latency, not the bandwidth, is what a per-chunk wait exposes),
+        // then the row max in eight independent chains
         float s[kBlockN];
         float mx[8];
         tmem_ld32(tS, s);
-        tmem_wait_ld_into(s);
         tmem_ld32(tS + 32, s + 32);
+        tmem_ld32(tS + 64, s + 64);
+        tmem_ld32(tS + 96, s + 96);
+        tmem_wait_ld_into(s);
+        tmem_tie32(s + 32);
+        tmem_tie32(s + 64);
+        tmem_tie32(s + 96);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          mx[i] = max3f(s[4 * i], s[4 * i + 1], fmaxf(s[4 * i + 2], s[4 * i + 3]));
+        for (int i = 0; i < 8; ++i) mx[i] = s[i];
 #pragma unroll
-        for (int c = 1; c < kBlockN / 32; ++c) {
-          tmem_wait_ld_into(s + 32 * c);
-          if (c + 1 < kBlockN / 32) tmem_ld32(tS + 32 * (c + 1), s + 32 * (c + 1));
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            mx[i] = max3f(mx[i], s[32 * c + 4 * i], s[32 * c + 4 * i + 1]);
-            mx[i] = max3f(mx[i], s[32 * c + 4 * i + 2], s[32 * c + 4 * i + 3]);
-          }
-        }
+        for (int c = 8; c < kBlockN; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
         const int valid = w.valid();
         if (valid < kBlockN) {
 #pragma unroll
@@ -566,7 +625,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_ready[t]);
+        named_arrive(kPBarBase + t, kPBarThreads);   // P_t of this warp is in tensor memory
         w.next(p);
       }
       if (!ok) break;

@@ -290,8 +290,36 @@ __device__ __forceinline__ void tmem_wait_ld_into(float* r) {
                :
                : "memory");
 }
+// Marks 32 registers as written at this point without an instruction: put
+// after a tmem_wait_ld_into() that also covered their load, so no use of
+// them is scheduled before that wait.
+__device__ __forceinline__ void tmem_tie32(float* r) {
+  asm volatile(""
+               : "+f"(r[0]), "+f"(r[1]), "+f"(r[2]), "+f"(r[3]), "+f"(r[4]), "+f"(r[5]),
+                 "+f"(r[6]), "+f"(r[7]), "+f"(r[8]), "+f"(r[9]), "+f"(r[10]), "+f"(r[11]),
+                 "+f"(r[12]), "+f"(r[13]), "+f"(r[14]), "+f"(r[15]), "+f"(r[16]), "+f"(r[17]),
+                 "+f"(r[18]), "+f"(r[19]), "+f"(r[20]), "+f"(r[21]), "+f"(r[22]), "+f"(r[23]),
+                 "+f"(r[24]), "+f"(r[25]), "+f"(r[26]), "+f"(r[27]), "+f"(r[28]), "+f"(r[29]),
+                 "+f"(r[30]), "+f"(r[31])
+               :
+               : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// ----------------------------------------------------------------- named barriers
+// Hardware CTA barriers 1..15 (0 is __syncthreads), counted in threads of
+// whole warps; every thread of a calling warp executes the instruction.
+// A producer warp arrives (never blocks); a consumer warp syncs (blocks
+// until `nthreads` threads have arrived or synced).  Arrive has release and
+// sync acquire semantics for the participating threads.  A named barrier
+// has no time limit: a kernel that syncs on one must guarantee the arrivals.
+__device__ __forceinline__ void named_arrive(uint32_t id, uint32_t nthreads) {
+  asm volatile("barrier.cta.arrive.aligned %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("barrier.cta.sync.aligned %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ----------------------------------------------------------------- descriptors
