@@ -19,3 +19,21 @@ def cuda_ok():
     if not torch.cuda.is_available():
         pytest.fail("gpu test run without a CUDA device")
     return True
+
+
+@pytest.fixture(autouse=True)
+def _device_error_word_clear(request):
+    """After every GPU test the library's device error word must be clear: no
+    bounded wait gave up and, on the bounds-checking build, no index check
+    fired.  Tests that provoke an error on purpose read (and so clear) the
+    word themselves."""
+    yield
+    if request.node.get_closest_marker("gpu") is None:
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    import context_attention_dits_cp_b200 as cp
+    from context_attention_dits_cp_b200 import binding as bd
+    st = cp.last_device_error()
+    assert st == 0, f"device error word after the test: {bd.STATUS.get(st, st)}"

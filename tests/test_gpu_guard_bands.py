@@ -248,14 +248,17 @@ def test_ulysses_anything_attention_stays_inside(cuda_ok, B):
     _no_device_error()
 
 
-@pytest.mark.skipif(os.environ.get("CPATTN_GUARD_CHILD") == "1",
-                    reason="the child runs the debug build")
+@pytest.mark.skipif(os.environ.get("CPATTN_GUARD_CHILD") == "1" or
+                    os.environ.get("CPATTN_DEBUG") == "1",
+                    reason="the bounds-checking build is loaded")
 def test_bounds_selftest_is_silent_in_the_release_build(cuda_ok):
     assert not cp.is_debug_build()
     assert cp.selftest_bounds_check() == 0
 
 
-@pytest.mark.skipif(os.environ.get("CPATTN_GUARD_CHILD") == "1", reason="no grandchildren")
+@pytest.mark.skipif(os.environ.get("CPATTN_GUARD_CHILD") == "1" or
+                    os.environ.get("CPATTN_DEBUG") == "1",
+                    reason="no grandchildren; the whole run already uses the bounds-checking build")
 def test_every_guard_band_again_on_the_bounds_checking_build(cuda_ok):
     """This file, rerun in a child process on libcpattn_debug.so: the checks
     are live (the self-test's deliberate failure is reported), and none of
