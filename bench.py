@@ -240,8 +240,18 @@ def run_cuda(args):
     flush_clean = lambda: (flush_buf.fill_(1), flush_buf.sum(dtype=torch.int32))
     step = lambda: cp.ring_attention(dq, dk, dv, offs, out=out, lse=lse)
     flops = w.flops
-    if args.profile_run in ("merge", "permute"):
-        if args.profile_run == "merge":
+    if args.profile_run in ("merge", "permute", "walk"):
+        if args.profile_run == "walk":
+            # the literal per-chunk ring step: chunk 0 alone, chunks 1.. merged in
+            kcs = [(dk[:, offs[c]:offs[c + 1]], dv[:, offs[c]:offs[c + 1]]) for c in range(len(offs) - 1)]
+            acc = torch.empty_like(out)
+            lacc = torch.empty_like(lse)
+
+            def fn():
+                cp.attn_partial(dq, *kcs[0], out=acc, lse=lacc)
+                for kc, vc in kcs[1:]:
+                    cp.attn_partial_merge(dq, kc, vc, acc, lacc)
+        elif args.profile_run == "merge":
             acc = torch.zeros_like(out)
             lacc = torch.full_like(lse, -float("inf"))
             oi = torch.randn(out.shape, device=dev)
@@ -782,7 +792,7 @@ def main():
     ap.add_argument("--extra", action="store_true", help="also time the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-run", nargs="?", const="ring", default=None,
-                    choices=("ring", "merge", "permute"),
+                    choices=("ring", "merge", "permute", "walk"),
                     help="only warm-up + timed launches of one kernel (for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
