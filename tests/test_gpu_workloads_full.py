@@ -5,6 +5,8 @@ times, compared element by element with the CPU fp64 oracle.
   literal per-chunk walk and the gathered Ring Anything layout) and both
   Ulysses / unified paths (R 1 x U 4 and R 2 x U 2): every query row of every
   head.
+* the head-dim-64 case the benchmark also times (FLUX token count, 48 heads
+  of 64): every row of every head.
 * high-res 16k (8 chunks, +-8 outliers) and video 32761 (7 x 4096 + 4089):
   the oracle would need minutes for every row, so each head is checked on a
   seeded stratified sample -- four rows in every 128-row query tile (16k),
@@ -197,3 +199,15 @@ def test_ulysses_and_unified_every_row(cuda_ok, R, U):
     del out
     ro, rl = _full_reference(w.name)
     check(o_full, lse.cpu(), ro, rl, torch.bfloat16)
+
+
+# ---------------------------------------------------------------- head dim 64
+def test_head_dim_64_flux_tokens_every_row(cuda_ok):
+    """The benchmark's head-dim-64 case: the FLUX token count (4608, four
+    chunks of 1152) with 48 heads of 64, every row of every head."""
+    q, k, v = wl.make_qkv(1, 48, 4608, 64, torch.bfloat16, 1201, "kscale")
+    offs = wl.chunk_offsets(wl.ring_chunk_lengths(4608, 4))
+    out, lse = cp.ring_attention(q.cuda(), k.cuda(), v.cuda(), offs)
+    torch.cuda.synchronize()
+    ro, rl = oracle_by_head(_np(q), _np(k), _np(v))
+    check(out, lse, ro, rl, torch.bfloat16)
