@@ -1,8 +1,9 @@
 """The five workloads at full size, in the launch configuration the benchmark
 times, compared element by element with the CPU fp64 oracle.
 
-* tiny ring (fp32, 2 chunks), FLUX joint attention (the plain ring walk, the
-  literal per-chunk walk and the gathered Ring Anything layout) and both
+* tiny ring (fp32, 2 chunks), FLUX joint attention (the plain ring walk with
+  fp32 and with bf16 output, the literal per-chunk walk and the gathered Ring
+  Anything layout) and both
   Ulysses / unified paths (R 1 x U 4 and R 2 x U 2): every query row of every
   head.
 * the head-dim-64 case the benchmark also times (FLUX token count, 48 heads
@@ -137,6 +138,19 @@ def test_flux_ring4_every_row(cuda_ok):
     offs = wl.chunk_offsets(wl.ring_chunk_lengths(w.S, w.ring_degree))
     out, lse = cp.ring_attention(q.cuda(), k.cuda(), v.cuda(), offs)
     torch.cuda.synchronize()
+    ro, rl = _full_reference(w.name)
+    check(out, lse, ro, rl, w.torch_dtype)
+
+
+def test_flux_ring4_bf16_out_every_row(cuda_ok):
+    """The same walk with the output cast to bf16 in the epilogue (lse stays
+    fp32); the cast adds at most half a bf16 ulp of |out| to the error."""
+    w, q, k, v = _inputs("flux_joint_ring4")
+    offs = wl.chunk_offsets(wl.ring_chunk_lengths(w.S, w.ring_degree))
+    out = torch.empty((w.B, w.S, w.H, w.D), dtype=torch.bfloat16, device="cuda")
+    out, lse = cp.ring_attention(q.cuda(), k.cuda(), v.cuda(), offs, out=out)
+    torch.cuda.synchronize()
+    assert out.dtype == torch.bfloat16
     ro, rl = _full_reference(w.name)
     check(out, lse, ro, rl, w.torch_dtype)
 
